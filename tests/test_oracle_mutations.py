@@ -1,0 +1,85 @@
+"""The oracle's pins are strong enough to catch plausible mistakes.
+
+Each case plants one mistake in a temporary copy of oracle.c (on the CPU),
+builds it, runs the pin suite against that build and expects at least one
+pin to fail.  The real oracle is untouched.
+"""
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+import tests.test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "oracle.c")
+
+MUTANTS = {
+    "relu_dropped": ("double relu = dot > 0.0 ? dot : 0.0;", "double relu = dot;"),
+    "w_wrong_head": ("I += (double)w[(int64_t)t * HI + h] * relu;", "I += (double)w[(int64_t)t * HI] * relu;"),
+    "k_dims_shifted": ("dot += q[h * DI + d] * orc_e4m3_to_f64(k[d]);",
+                       "dot += q[h * DI + d] * orc_e4m3_to_f64(k[(d + 1) % DI]);"),
+    "q_head_transposed": ("dot += q[h * DI + d] * orc_e4m3_to_f64(k[d]);",
+                          "dot += q[d * HI % (HI * DI) + h] * orc_e4m3_to_f64(k[d]);"),
+    "causal_off_by_one": ("for (int64_t s = 0; s <= p; ++s) {", "for (int64_t s = 0; s < p; ++s) {"),
+    "page_table_ignored": ("return (int64_t)page * page_size + pos % page_size;",
+                           "return lp * page_size + pos % page_size;"),
+    "tie_to_higher_pos": ("return (x->pos < y->pos) ? -1 : (x->pos > y->pos);",
+                          "return (x->pos > y->pos) ? -1 : (x->pos < y->pos);"),
+    "ascending_scores": ("if (x->v > y->v) return -1;\n    if (x->v < y->v) return 1;",
+                         "if (x->v < y->v) return -1;\n    if (x->v > y->v) return 1;"),
+    "gate_dropped": ("for (int d = 0; d < Dv; ++d) o[d] *= sig;", "for (int d = 0; d < Dv; ++d) o[d] *= 1.0;"),
+    "gate_not_sigmoid": ("double sig = 1.0 / (1.0 + exp(-g));", "double sig = g;"),
+    "scale_dropped": ("lg[j] = sm_scale * dot;", "lg[j] = dot;"),
+    "value_rows_shifted": ("for (int d = 0; d < Dv; ++d) o[d] += p * orc_bf16_to_f64(c[d]);",
+                           "for (int d = 0; d < Dv; ++d) o[d] += p * orc_bf16_to_f64(c[Dqk - Dv + d]);"),
+    "e4m3_bias": ("else        v = ldexp(1.0 + (double)m / 8.0, e - 7);",
+                  "else        v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    "swa_window_short": ("int64_t p0 = L - W > 0 ? L - W : 0;", "int64_t p0 = L - W + 1 > 0 ? L - W + 1 : 0;"),
+    "swa_wrong_slot": ("int64_t slot = (p0 + i) % W;\n                const uint16_t *k",
+                       "int64_t slot = i % W;\n                const uint16_t *k"),
+}
+
+PIN_TESTS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]
+
+
+def _pin_failures(orc):
+    failed = []
+    for fn in PIN_TESTS:
+        args = {}
+        import inspect
+        params = inspect.signature(fn).parameters
+        if "orc" in params:
+            args["orc"] = orc
+        if "kind" in params:
+            for kind in ("normal", "ties", "zeros", "const", "dyadic"):
+                try:
+                    fn(orc=orc, kind=kind)
+                except Exception:
+                    failed.append(f"{fn.__name__}[{kind}]")
+            continue
+        try:
+            fn(**args)
+        except Exception:
+            failed.append(fn.__name__)
+    return failed
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(orc, name):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor for {name} not found"
+    mutated = src.replace(old, new, 1)
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "m.c")
+        so = os.path.join(d, "m.so")
+        open(c, "w").write(mutated)
+        subprocess.check_call(["gcc", "-O1", "-fopenmp", "-shared", "-fPIC", "-std=c11", "-o", so, c, "-lm"])
+        with orc.use_library(so):
+            failed = _pin_failures(orc)
+    assert failed, f"no pin caught the planted mistake '{name}'"
+
+
+def test_unmutated_oracle_passes_every_pin(orc):
+    assert _pin_failures(orc) == []
