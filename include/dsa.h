@@ -1,0 +1,188 @@
+/*
+ * dsa.h -- C ABI of libdsa.so, a B200 (sm_100a) implementation of the Gated
+ * DeepSeek Sparse Attention (DSA) layer.
+ *
+ * The layer, as the source pages describe it, has three stages, run in this
+ * order for every query token:
+ *   1. a lightweight multi-head indexer without rotary embedding scores every
+ *      causal history position ("Open-Source LLM Architecture Evolution: How
+ *      Lightweight Sparse Attention Reshapes Long-Context Modeling Efficiency",
+ *      Architecture Breakdown §2, "Indexer"; "Fine-Grained Sparse Attention in
+ *      Ultra-Large Parameter Models", §2.1-§2.3);
+ *   2. top-K selection keeps the K = 2048 best positions (same page, "Top-K
+ *      selection"; "Open-Sourcing Ultra-Large Sparse Attention Models", §2.2);
+ *   3. attention and softmax over only the selected positions ("Open-Source
+ *      LLM Architecture Evolution", Technical Deep Dive §2), its output scaled
+ *      by a gate ("Gated fusion"; read here as a per-head sigmoid gate).
+ * No page writes a formula; this library fixes the score as
+ *   I[t,s] = sum_h w[t,h] * ReLU(qI[t,h,:] . kI[s,:])
+ * and breaks top-K ties toward the lower position.
+ *
+ * Conventions (every entry point):
+ *  - Pointers marked "device" are CUDA device memory allocated and owned by
+ *    the caller; the library never allocates, frees or retains them.
+ *  - 8-bit floats are OCP E4M3 ("e4m3fn") bytes; bf16 values travel as their
+ *    16-bit patterns (uint16_t).  All arrays are dense row-major.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and the call returns without synchronising.  Argument checks
+ *    that need only host data run first; on failure nothing is launched.
+ *  - Device-side checks (positions past a sequence, page ids out of range,
+ *    a pipeline wait that exceeds its time limit) skip the offending access
+ *    and set bits in a per-device error word read by dsa_device_error().
+ *  - Calls are thread-safe; calls on one stream run in order.
+ *  - Shapes outside the supported set return DSA_ERR_UNSUPPORTED; there is no
+ *    fallback path.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSA_ABI_VERSION 1
+
+typedef struct CUstream_st *dsa_stream_t; /* same handle as cudaStream_t */
+
+typedef enum {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned buffer */
+    DSA_ERR_UNSUPPORTED = 2, /* shape outside the tuned set */
+    DSA_ERR_WORKSPACE = 3,   /* workspace missing or too small */
+    DSA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+    DSA_ERR_TIMEOUT = 5      /* reported through dsa_device_error() only */
+} dsa_status;
+
+/* Device error word bits (dsa_device_error). */
+#define DSA_DEVERR_POSITION 0x1u  /* q_pos/idx outside its sequence: row skipped */
+#define DSA_DEVERR_PAGE 0x2u      /* block-table entry outside [0, num_pages) */
+#define DSA_DEVERR_TIMEOUT 0x4u   /* a pipeline wait hit its time limit */
+#define DSA_DEVERR_SHAPE 0x8u     /* a per-row length exceeded its host bound */
+
+/* Paged cache geometry.  A cache is [num_pages, page_size, row] and sequence
+ * b's logical position p lives in physical page block_table[b][p / page_size],
+ * row p % page_size.  page_size must be 64. */
+typedef struct {
+    const int32_t *seq_lens;    /* device [num_seqs]: tokens in each sequence */
+    const int32_t *block_table; /* device [num_seqs, max_blocks_per_seq] */
+    int32_t num_seqs;
+    int32_t max_blocks_per_seq;
+    int32_t page_size;
+    int32_t num_pages;
+} dsa_paged;
+
+/* ---- stage 1: indexer scores ------------------------------------------
+ * scores[t*ld + s] = sum_h w[t*HI + h] * max(0, sum_d qI[t,h,d] * kI(q_seq[t], s)[d])
+ * for 0 <= s <= q_pos[t], where kI(b, s) is row s of sequence b in the paged
+ * indexer-key cache.  Scores are fp32 (FP8 products accumulate in fp32);
+ * entries s > q_pos[t] are not written.
+ *   q_idx       device e4m3 [T, HI, DI]
+ *   w           device fp32 [T, HI]    (any sign; model scales folded in)
+ *   k_idx_cache device e4m3 [num_pages, 64, DI]; base 16-byte aligned
+ *   q_seq,q_pos device int32 [T]; NULL for both means decode: query t is the
+ *               last token of sequence t (T == num_seqs, q_pos = seq_len-1)
+ *   max_len     host bound: every q_pos[t] < max_len <= ld
+ *   scores      device fp32 [T, ld]
+ * Supported: HI in {4, 8, 16, 32, 64}, DI in {64, 128}.  Needs no workspace. */
+dsa_status dsa_indexer_scores(const uint8_t *q_idx, const float *w,
+                              const uint8_t *k_idx_cache, const dsa_paged *pg,
+                              const int32_t *q_seq, const int32_t *q_pos,
+                              int32_t T, int32_t HI, int32_t DI, int32_t max_len,
+                              float *scores, int64_t ld, dsa_stream_t stream);
+
+/* ---- stage 2: top-K --------------------------------------------------------
+ * For each row r: among positions 0 <= s < row_len[r], keep the K largest
+ * scores[r*ld + s] under the order (score descending, position ascending),
+ * with -0.0 equal to +0.0.  A row with row_len[r] <= K keeps every position.
+ * idx[r*K + j] receives the kept positions in ascending order, then -1.
+ * Scores must be finite.
+ *   row_len     device int32 [R]; every row_len[r] <= max_row_len <= ld
+ *   idx         device int32 [R, K]
+ *   ws          device scratch of dsa_topk_workspace_bytes(R, K, max_row_len)
+ *               bytes, 256-byte aligned; contents need no initialisation.
+ * Supported: 1 <= K <= 4096. */
+size_t dsa_topk_workspace_bytes(int32_t R, int32_t K, int32_t max_row_len);
+dsa_status dsa_topk(const float *scores, int64_t ld, const int32_t *row_len,
+                    int32_t R, int32_t K, int32_t max_row_len, int32_t *idx,
+                    void *ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* ---- stage 3: gated attention over the selected latent rows ----------------
+ * For query t, head h, and the selected rows c_j = latent row idx[t*K + j] of
+ * sequence q_seq[t] (entries < 0 are padding):
+ *   l_j = sm_scale * (q[t,h,:Dqk] . c_j[:Dqk]),  p = softmax_j(l),
+ *   out[t,h,:] = bf16( sigmoid(gate[t,h]) * sum_j p_j c_j[:Dv] ).
+ * All H heads share the latent row (key = its first Dqk entries, value = its
+ * first Dv).  A query with no valid entry gets out = 0 (and lse = -inf).
+ *   q        device bf16 [T, H, Dqk]; kv_cache device bf16 [num_pages, 64, Dqk]
+ *   q_seq    device int32 [T], or NULL for decode (query t -> sequence t)
+ *   gate     device bf16 [T, H];  out device bf16 [T, H, Dv]
+ *   lse      device fp32 [T, H] or NULL: natural-log sum of exp(l_j)
+ *   ws       dsa_sparse_attn_workspace_bytes(T, H, K, Dv) bytes (may be 0)
+ * Supported: (Dqk, Dv) in {(576, 512), (64, 64)}, 1 <= H <= 128,
+ * K a multiple of 64, K <= 4096.  Buffers 16-byte aligned. */
+size_t dsa_sparse_attn_workspace_bytes(int32_t T, int32_t H, int32_t K, int32_t Dv);
+dsa_status dsa_sparse_attn(const uint16_t *q, const uint16_t *kv_cache,
+                           const dsa_paged *pg, const int32_t *q_seq,
+                           const int32_t *idx, int32_t K, const uint16_t *gate,
+                           float sm_scale, int32_t T, int32_t H, int32_t Dqk,
+                           int32_t Dv, uint16_t *out, float *lse, void *ws,
+                           size_t ws_bytes, dsa_stream_t stream);
+
+/* ---- the layer ----------------------------------------------------------------
+ * Runs stage 1 -> 2 -> 3 on one stream.  Prefill: T query tokens with explicit
+ * q_seq/q_pos.  Decode: one query per sequence at position seq_len-1
+ * (q_seq/q_pos ignored, T == pg.num_seqs).  Row t's candidate count is
+ * q_pos[t] + 1. */
+enum { DSA_MODE_PREFILL = 0, DSA_MODE_DECODE = 1 };
+
+typedef struct {
+    int32_t mode;
+    const uint8_t *q_idx;       /* device e4m3 [T, HI, DI] */
+    const float *w;             /* device fp32 [T, HI] */
+    const uint8_t *k_idx_cache; /* device e4m3 [num_pages, 64, DI] */
+    const uint16_t *q;          /* device bf16 [T, H, Dqk] */
+    const uint16_t *kv_cache;   /* device bf16 [num_pages, 64, Dqk] */
+    const uint16_t *gate;       /* device bf16 [T, H] */
+    dsa_paged pg;
+    const int32_t *q_seq;       /* device int32 [T] (prefill) */
+    const int32_t *q_pos;       /* device int32 [T] (prefill) */
+    int32_t T, HI, DI, K, H, Dqk, Dv;
+    int32_t max_len;            /* host bound on q_pos+1 (prefill) / seq_lens (decode) */
+    float sm_scale;
+    uint16_t *out;              /* device bf16 [T, H, Dv] */
+    int32_t *idx_out;           /* device int32 [T, K] or NULL */
+    float *lse;                 /* device fp32 [T, H] or NULL */
+} dsa_layer_args;
+
+/* Workspace: fp32 scores [T, max_len] + top-K scratch (+ idx if idx_out is
+ * NULL) + split-K attention partials. */
+size_t dsa_layer_workspace_bytes(const dsa_layer_args *a);
+dsa_status dsa_layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes,
+                             dsa_stream_t stream);
+
+/* ---- sliding-window decode (the hybrid's local layers) ------------------------
+ * "aiany.app item naive-n0-5-flash", Key Capabilities: 5 sliding-window
+ * layers (window 128) per DSA layer.  Sequence b's query (position
+ * L-1, L = seq_lens[b]) attends causally to positions [max(0, L-window), L-1],
+ * stored in ring slot p % window; multi-head with H K/V heads.
+ *   q device bf16 [B, H, D]; k_ring, v_ring device bf16 [B, window, H, D];
+ *   out device bf16 [B, H, D].  Supported: D == 128, window == 128, H % 8 == 0. */
+dsa_status dsa_swa_decode(const uint16_t *q, const uint16_t *k_ring,
+                          const uint16_t *v_ring, const int32_t *seq_lens,
+                          int32_t B, int32_t H, int32_t D, int32_t window,
+                          float sm_scale, uint16_t *out, dsa_stream_t stream);
+
+/* ---- housekeeping ---------------------------------------------------------------- */
+const char *dsa_status_string(dsa_status s);
+int32_t dsa_abi_version(void);
+/* Synchronously reads (and, if reset != 0, clears) the current device's error
+ * word; *code receives DSA_DEVERR_* bits, 0 when all is well. */
+dsa_status dsa_device_error(uint32_t *code, int32_t reset);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DSA_H_ */

@@ -1,0 +1,543 @@
+// Stage 3 of the Gated DSA layer: attention over only the selected latent
+// rows, multiplied by a per-head sigmoid gate.
+//
+// ("Open-Source LLM Architecture Evolution", Technical Deep Dive §2: scores
+// and softmax over only the 2048 selected elements; Architecture Breakdown
+// §2, "Gated fusion", read as out = sigmoid(g) * attention output.)  All
+// heads share the selected latent row: the key is its first Dqk entries and
+// the value its first Dv.
+//
+// One CTA = (query token, a 256-wide slice of the value dims, a split of the
+// selected rows).  The selected rows are gathered 64 at a time through the
+// block table with 16-byte async copies straight into the 128-byte-swizzled
+// layout the tensor core reads; Q arrives by TMA.  tcgen05 bf16 MMAs compute
+// S = Q C^T (M = 128 heads, N = 64 rows, fp32 in TMEM, double-buffered) and
+// O += P V (V read as an MN-major operand from the same gathered tile); the
+// softmax warps keep the running max in the exp2 domain and rescale O in
+// TMEM only when the max grows by more than 2^8.  With one split the gate is
+// applied in the epilogue; otherwise normalised partials and (max, sum) go
+// to the workspace and attn_combine_kernel merges them and applies the gate.
+//
+// Warps 0-3: softmax/epilogue (one TMEM lane quarter each, a thread per
+// head); warp 4: MMA issuer and TMEM owner; warps 5-8: gather producers.
+#include "dsa_device.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+namespace {
+
+constexpr int ATT_THREADS = 288;
+
+template <int DQK, int DVP>
+struct AttnCfg {
+    static constexpr int KQ = DQK / 64;   // 128-byte k-blocks of a latent row used by S
+    static constexpr int NVB = DVP / 64;  // 64-dim value blocks per CTA
+    static constexpr int NC = 64;         // selected rows per chunk
+    static constexpr int NST = 8;         // gather ring stages
+    static constexpr int LAG = 4;         // copies a producer keeps in flight before signalling
+    static constexpr int STAGE_BYTES = NC * 128;
+    static constexpr int Q_BYTES = KQ * 128 * 128;
+    static constexpr int P_BYTES = 128 * 128;
+    static constexpr int S_COL = 0;
+    static constexpr int O_COL = 128;
+    static constexpr int TMEM_COLS = (O_COL + DVP) <= 256 ? 256 : 512;
+    static constexpr int NBAR = 2 * NST + 8;
+    static constexpr int SMEM = 1024 + Q_BYTES + NST * STAGE_BYTES + P_BYTES + 8 * NBAR + 64;
+    static_assert(DQK % 64 == 0 && DVP % 64 == 0 && DVP <= DQK, "shape");
+};
+
+struct AttnParams {
+    const uint16_t *kv;
+    PagedDev pg;
+    const int32_t *q_seq;
+    const int32_t *idx;
+    int32_t K;
+    const uint16_t *gate;
+    float scale_log2;
+    int32_t T, H, Dv, nparts, splits, rows_per_split;
+    uint16_t *out;
+    float *lse;
+    float *part_o;   // [T, splits, H, Dv] normalised partial outputs
+    float *part_ml;  // [T, splits, H, 2]   (running max in log2 units, sum)
+    uint32_t *err;
+};
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Latent-cache row of selected entry g of token t, or -1 when the entry is
+// padding, past the split, or invalid (recorded when `report`).
+__device__ __forceinline__ int64_t latent_row(const AttnParams &p, int b, int L, int t, int g, int row_end,
+                                              bool report) {
+    if (g >= row_end) return -1;
+    const int pos = p.idx[(int64_t)t * p.K + g];
+    if (pos < 0) return -1;
+    if (pos >= L) {
+        if (report) record_error(p.err, DSA_DEVERR_POSITION);
+        return -1;
+    }
+    const int lp = pos >> 6;
+    if (lp >= p.pg.max_blocks) {
+        if (report) record_error(p.err, DSA_DEVERR_PAGE);
+        return -1;
+    }
+    const int pg = p.pg.block_table[(int64_t)b * p.pg.max_blocks + lp];
+    if (pg < 0 || pg >= p.pg.num_pages) {
+        if (report) record_error(p.err, DSA_DEVERR_PAGE);
+        return -1;
+    }
+    return (int64_t)pg * 64 + (pos & 63);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+template <int DQK, int DVP>
+__global__ void __launch_bounds__(ATT_THREADS, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap qmap, const AttnParams p) {
+    using C = AttnCfg<DQK, DVP>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    uint8_t *Qs = smem;
+    uint8_t *ring = Qs + C::Q_BYTES;
+    uint8_t *Ps = ring + C::NST * C::STAGE_BYTES;
+    uint64_t *full = reinterpret_cast<uint64_t *>(Ps + C::P_BYTES);
+    uint64_t *empty = full + C::NST;
+    uint64_t *q_full = empty + C::NST;
+    uint64_t *s_full = q_full + 1;   // [2]
+    uint64_t *s_empty = s_full + 2;  // [2]
+    uint64_t *p_full = s_empty + 2;
+    uint64_t *o_done = p_full + 1;
+    uint64_t *drain = o_done + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    int *last_sh = reinterpret_cast<int *>(tmem_slot + 1);
+    volatile int *abort_flag = last_sh + 1;
+
+    const int warp = warp_id(), lane = lane_id();
+    const int t = blockIdx.y;
+    const int part = blockIdx.x % p.nparts;
+    const int split = blockIdx.x / p.nparts;
+    const int row0 = split * p.rows_per_split;
+    const int row_end = min(p.K, row0 + p.rows_per_split);
+
+    int b = p.q_seq ? p.q_seq[t] : t;
+    bool tok_ok = b >= 0 && b < p.pg.num_seqs;
+    const int L = tok_ok ? p.pg.seq_lens[b] : 0;
+    if (!tok_ok) b = 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::NST; ++s) {
+            mbar_init(&full[s], 128);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_empty[i], 4);
+        }
+        mbar_init(p_full, 4);
+        mbar_init(o_done, 1);
+        mbar_init(drain, 1);
+        *last_sh = -1;
+        *abort_flag = 0;
+        if (!tok_ok) record_error(p.err, DSA_DEVERR_POSITION);
+        fence_mbar_init();
+        tma_prefetch_desc(&qmap);
+    }
+    if (warp == 4) tmem_alloc(tmem_slot, C::TMEM_COLS);
+    __syncthreads();
+    if (tok_ok)
+        for (int g = row0 + threadIdx.x; g < row_end; g += ATT_THREADS)
+            if (p.idx[(int64_t)t * p.K + g] >= 0) atomicMax(last_sh, g);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int nc = *last_sh < 0 ? 0 : (*last_sh - row0) / C::NC + 1;
+
+    if (warp >= 5) {
+        // ---------------- gather producers ----------------
+        const int pi = threadIdx.x - 160;
+        const int r = pi >> 1, half = pi & 1;
+        if (pi == 0 && nc > 0) {
+            mbar_expect_tx(q_full, C::Q_BYTES);
+            for (int kb = 0; kb < C::KQ; ++kb) tma_load_2d(Qs + kb * 128 * 128, &qmap, q_full, kb * 64, t * p.H);
+        }
+        int ld = 0;
+        bool ok = true;
+        int64_t src_cur = -1, src_prev = -1;
+        auto load_block = [&](int bi, int64_t src) -> bool {
+            const int s = ld % C::NST;
+            if (!mbar_wait(&empty[s], ((ld / C::NST) & 1) ^ 1, p.err, abort_flag)) return false;
+            uint8_t *dst = ring + s * C::STAGE_BYTES + r * 128;
+            const uint16_t *g = p.kv + src * DQK + bi * 64;
+#pragma unroll
+            for (int cc = half * 4; cc < half * 4 + 4; ++cc) {
+                uint8_t *d = dst + ((cc ^ (r & 7)) << 4);
+                if (src >= 0) cp_async_16(d, g + cc * 8);
+                else *reinterpret_cast<uint4 *>(d) = make_uint4(0, 0, 0, 0);
+            }
+            cp_async_commit();
+            if (ld >= C::LAG) {
+                cp_async_wait<C::LAG>();
+                fence_proxy_async_smem();
+                mbar_arrive(&full[(ld - C::LAG) % C::NST]);
+            }
+            ++ld;
+            return true;
+        };
+        for (int c = 0; ok && c <= nc; ++c) {
+            if (c < nc) {
+                src_cur = latent_row(p, b, L, t, row0 + c * C::NC + r, row_end, half == 0);
+                for (int kb = 0; ok && kb < C::KQ; ++kb) ok = load_block(kb, src_cur);
+            }
+            if (c >= 1)
+                for (int db = 0; ok && db < C::NVB; ++db) ok = load_block(part * C::NVB + db, src_prev);
+            src_prev = src_cur;
+        }
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        if (ok)
+            for (int i = ld - C::LAG < 0 ? 0 : ld - C::LAG; i < ld; ++i) mbar_arrive(&full[i % C::NST]);
+        if (pi == 0 && nc > 0) mbar_wait(q_full, 0, p.err, nullptr);
+    } else if (warp == 4) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0 && nc > 0) {
+            constexpr uint32_t ID_S = idesc(1, 1, 0, 0, C::NC, 128);
+            constexpr uint32_t ID_PV = idesc(1, 1, 0, 1, 64, 128);
+            bool ok = mbar_wait(q_full, 0, p.err, abort_flag);
+            tc_fence_after();
+            const uint32_t qa0 = smem_u32(Qs), ring0 = smem_u32(ring), pa = smem_u32(Ps);
+            int ld = 0;
+            for (int c = 0; ok && c <= nc; ++c) {
+                if (c < nc) {
+                    const int sb = c & 1;
+                    if (!mbar_wait(&s_empty[sb], ((c >> 1) & 1) ^ 1, p.err, abort_flag)) break;
+                    tc_fence_after();
+                    const uint32_t dS = tmem + C::S_COL + sb * C::NC;
+                    for (int kb = 0; ok && kb < C::KQ; ++kb) {
+                        const int s = ld % C::NST;
+                        if (!mbar_wait(&full[s], (ld / C::NST) & 1, p.err, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t qa = qa0 + kb * 128 * 128, ca = ring0 + s * C::STAGE_BYTES;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            mma_bf16(dS, sdesc(qa + 32 * k, 16, 1024, SWZ_128B), sdesc(ca + 32 * k, 16, 1024, SWZ_128B),
+                                     ID_S, (kb | k) != 0);
+                        mma_commit(&empty[s]);
+                        ++ld;
+                    }
+                    if (!ok) break;
+                    mma_commit(&s_full[sb]);
+                }
+                if (c >= 1) {
+                    const int j = c - 1;
+                    if (!mbar_wait(p_full, j & 1, p.err, abort_flag)) break;
+                    tc_fence_after();
+                    for (int db = 0; ok && db < C::NVB; ++db) {
+                        const int s = ld % C::NST;
+                        if (!mbar_wait(&full[s], (ld / C::NST) & 1, p.err, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t ca = ring0 + s * C::STAGE_BYTES;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            mma_bf16(tmem + C::O_COL + db * 64, sdesc(pa + 32 * k, 16, 1024, SWZ_128B),
+                                     sdesc(ca + 2048 * k, C::STAGE_BYTES, 1024, SWZ_128B), ID_PV, (j > 0 || k > 0));
+                        mma_commit(&empty[s]);
+                        ++ld;
+                    }
+                    if (!ok) break;
+                    mma_commit(o_done);
+                }
+            }
+            mma_commit(drain);
+            mbar_wait(drain, 0, p.err, nullptr);
+        }
+    } else {
+        // ---------------- softmax + epilogue (warps 0..3, thread = head) ----------------
+        const int row = threadIdx.x;  // 0..127
+        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        float m = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int c = 0; c < nc; ++c) {
+            const int sb = c & 1;
+            if (!mbar_wait(&s_full[sb], (c >> 1) & 1, p.err, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t sr[C::NC];
+            tmem_ld32(tmem + C::S_COL + sb * C::NC + lane_off, sr);
+            tmem_ld32(tmem + C::S_COL + sb * C::NC + 32 + lane_off, sr + 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[sb]);
+            const int gbase = row0 + c * C::NC;
+            const uint32_t vlo = __ballot_sync(0xffffffffu, latent_row(p, b, L, t, gbase + lane, row_end, false) >= 0);
+            const uint32_t vhi =
+                __ballot_sync(0xffffffffu, latent_row(p, b, L, t, gbase + 32 + lane, row_end, false) >= 0);
+            float x[C::NC];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < C::NC; ++i) {
+                const bool v = ((i < 32 ? vlo >> i : vhi >> (i - 32)) & 1u) != 0;
+                x[i] = v ? __uint_as_float(sr[i]) * p.scale_log2 : -INFINITY;
+                mx = fmaxf(mx, x[i]);
+            }
+            const float m_new = fmaxf(m, mx);
+            const bool resc = m_new > m + 8.f;
+            float alpha = 1.f;
+            if (resc) {
+                alpha = exp2f(m - m_new);
+                l *= alpha;
+                m = m_new;
+            }
+            uint32_t pk[C::NC / 2];
+            float lsum = 0.f;
+#pragma unroll
+            for (int i = 0; i < C::NC; i += 2) {
+                const float p0 = x[i] == -INFINITY ? 0.f : exp2f(x[i] - m);
+                const float p1 = x[i + 1] == -INFINITY ? 0.f : exp2f(x[i + 1] - m);
+                pk[i / 2] = pack_bf16(p0, p1);
+                const __nv_bfloat162 bv = *reinterpret_cast<__nv_bfloat162 *>(&pk[i / 2]);
+                lsum += __bfloat162float(bv.x) + __bfloat162float(bv.y);
+            }
+            l += lsum;
+            if (c >= 1) {
+                if (!mbar_wait(o_done, (c - 1) & 1, p.err, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (resc) {
+#pragma unroll 1
+                    for (int cc = 0; cc < DVP / 32; ++cc) {
+                        uint32_t o[32];
+                        const uint32_t ta = tmem + C::O_COL + cc * 32 + lane_off;
+                        tmem_ld32(ta, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32(ta, o);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            uint8_t *prow = Ps + row * 128;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc)
+                *reinterpret_cast<uint4 *>(prow + ((cc ^ (row & 7)) << 4)) =
+                    make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+        }
+        if (ok && nc > 0) ok = mbar_wait(o_done, (nc - 1) & 1, p.err, abort_flag);
+        tc_fence_after();
+        const bool have_o = ok && nc > 0;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const bool live = row < p.H;
+        if (p.splits == 1) {
+            const float g = live ? __bfloat162float(__ushort_as_bfloat16(p.gate[(int64_t)t * p.H + row])) : 0.f;
+            const float sig = 1.f / (1.f + __expf(-g));
+            const float scale = inv * sig;
+            uint16_t *orow = p.out + ((int64_t)t * p.H + row) * p.Dv + part * DVP;
+#pragma unroll 1
+            for (int cc = 0; cc < DVP / 32; ++cc) {
+                uint32_t o[32];
+                if (have_o) {
+                    tmem_ld32(tmem + C::O_COL + cc * 32 + lane_off, o);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = 0u;
+                }
+                if (live) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        uint4 v;
+                        v.x = pack_bf16(__uint_as_float(o[i]) * scale, __uint_as_float(o[i + 1]) * scale);
+                        v.y = pack_bf16(__uint_as_float(o[i + 2]) * scale, __uint_as_float(o[i + 3]) * scale);
+                        v.z = pack_bf16(__uint_as_float(o[i + 4]) * scale, __uint_as_float(o[i + 5]) * scale);
+                        v.w = pack_bf16(__uint_as_float(o[i + 6]) * scale, __uint_as_float(o[i + 7]) * scale);
+                        *reinterpret_cast<uint4 *>(orow + cc * 32 + i) = v;
+                    }
+                }
+            }
+            if (live && part == 0 && p.lse)
+                p.lse[(int64_t)t * p.H + row] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        } else {
+            const int64_t prow = ((int64_t)t * p.splits + split) * p.H + row;
+            float *po = p.part_o + prow * p.Dv + part * DVP;
+#pragma unroll 1
+            for (int cc = 0; cc < DVP / 32; ++cc) {
+                uint32_t o[32];
+                if (have_o) {
+                    tmem_ld32(tmem + C::O_COL + cc * 32 + lane_off, o);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = 0u;
+                }
+                if (live) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4 *>(po + cc * 32 + i) =
+                            make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
+                                        __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+                }
+            }
+            if (live && part == 0) {
+                p.part_ml[prow * 2 + 0] = m;
+                p.part_ml[prow * 2 + 1] = have_o ? l : 0.f;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// Merges split partials: out = sigmoid(g) * sum_s w_s o_s with
+// w_s = l_s 2^(m_s - M) / sum_s' l_s' 2^(m_s' - M).
+__global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
+    const int t = blockIdx.x;
+    const int h = blockIdx.y * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (h >= p.H) return;
+    const int S = p.splits;
+    float M = -INFINITY;
+    for (int s = 0; s < S; ++s) {
+        const float *ml = p.part_ml + (((int64_t)t * S + s) * p.H + h) * 2;
+        if (ml[1] > 0.f) M = fmaxf(M, ml[0]);
+    }
+    float wsum = 0.f;
+    for (int s = 0; s < S; ++s) {
+        const float *ml = p.part_ml + (((int64_t)t * S + s) * p.H + h) * 2;
+        if (ml[1] > 0.f) wsum += ml[1] * exp2f(ml[0] - M);
+    }
+    const float g = __bfloat162float(__ushort_as_bfloat16(p.gate[(int64_t)t * p.H + h]));
+    const float sig = 1.f / (1.f + __expf(-g));
+    const float inv = wsum > 0.f ? sig / wsum : 0.f;
+    uint16_t *orow = p.out + ((int64_t)t * p.H + h) * p.Dv;
+    for (int d0 = lane * 4; d0 < p.Dv; d0 += 128) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < S; ++s) {
+            const int64_t prow = ((int64_t)t * S + s) * p.H + h;
+            const float *ml = p.part_ml + prow * 2;
+            if (!(ml[1] > 0.f)) continue;
+            const float c = ml[1] * exp2f(ml[0] - M);
+            const float4 v = *reinterpret_cast<const float4 *>(p.part_o + prow * p.Dv + d0);
+            acc.x = fmaf(c, v.x, acc.x);
+            acc.y = fmaf(c, v.y, acc.y);
+            acc.z = fmaf(c, v.z, acc.z);
+            acc.w = fmaf(c, v.w, acc.w);
+        }
+        uint2 o;
+        o.x = pack_bf16(acc.x * inv, acc.y * inv);
+        o.y = pack_bf16(acc.z * inv, acc.w * inv);
+        *reinterpret_cast<uint2 *>(orow + d0) = o;
+    }
+    if (lane == 0 && p.lse)
+        p.lse[(int64_t)t * p.H + h] = wsum > 0.f ? (M + __log2f(wsum)) * 0.69314718055994531f : -INFINITY;
+}
+
+struct Plan {
+    int nparts, splits, rows_per_split;
+};
+
+Plan plan_for(int T, int K, int Dv, int sm_count) {
+    Plan pl;
+    pl.nparts = Dv == 512 ? 2 : 1;
+    const int nchunks = K / 64;
+    int splits = 1;
+    const int base = T * pl.nparts;
+    if (base < sm_count) splits = sm_count / base;
+    if (splits > nchunks) splits = nchunks;
+    if (splits < 1) splits = 1;
+    const int cps = (nchunks + splits - 1) / splits;
+    pl.rows_per_split = cps * 64;
+    pl.splits = (nchunks + cps - 1) / cps;
+    return pl;
+}
+
+template <int DQK, int DVP>
+dsa_status run_attn(const CUtensorMap &qm, const AttnParams &p, cudaStream_t st) {
+    using C = AttnCfg<DQK, DVP>;
+    auto fn = attn_kernel<DQK, DVP>;
+    if (!ensure_smem(reinterpret_cast<const void *>(fn), C::SMEM)) return DSA_ERR_CUDA;
+    dim3 grid(p.nparts * p.splits, p.T);
+    fn<<<grid, ATT_THREADS, C::SMEM, st>>>(qm, p);
+    if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+    if (p.splits > 1) {
+        dim3 cg(p.T, (p.H + 7) / 8);
+        attn_combine_kernel<<<cg, 256, 0, st>>>(p);
+        if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+    }
+    return DSA_OK;
+}
+
+}  // namespace
+
+size_t attn_workspace_bytes(int32_t T, int32_t H, int32_t K, int32_t Dv) {
+    const DeviceInfo *dev = current_device();
+    if (!dev || T <= 0 || K < 64) return 0;
+    Plan pl = plan_for(T, K, Dv, dev->sm_count);
+    if (pl.splits == 1) return 0;
+    const size_t rows = (size_t)T * pl.splits * H;
+    return align_up(rows * Dv * 4, 256) + align_up(rows * 2 * 4, 256);
+}
+
+dsa_status launch_attn(const AttnArgs &a, cudaStream_t st) {
+    const DeviceInfo *dev = current_device();
+    if (!dev) return DSA_ERR_CUDA;
+    if (a.T == 0) return DSA_OK;
+    Plan pl = plan_for(a.T, a.K, a.Dv, dev->sm_count);
+    AttnParams p{};
+    p.kv = a.kv;
+    p.pg = a.pg;
+    p.q_seq = a.q_seq;
+    p.idx = a.idx;
+    p.K = a.K;
+    p.gate = a.gate;
+    p.scale_log2 = a.sm_scale * 1.4426950408889634f;
+    p.T = a.T;
+    p.H = a.H;
+    p.Dv = a.Dv;
+    p.nparts = pl.nparts;
+    p.splits = pl.splits;
+    p.rows_per_split = pl.rows_per_split;
+    p.out = a.out;
+    p.lse = a.lse;
+    p.err = dev->err;
+    if (pl.splits > 1) {
+        const size_t rows = (size_t)a.T * pl.splits * a.H;
+        const size_t need = align_up(rows * a.Dv * 4, 256) + align_up(rows * 2 * 4, 256);
+        if (!a.ws || a.ws_bytes < need) return DSA_ERR_WORKSPACE;
+        p.part_o = static_cast<float *>(a.ws);
+        p.part_ml = reinterpret_cast<float *>(static_cast<uint8_t *>(a.ws) + align_up(rows * a.Dv * 4, 256));
+    }
+    CUtensorMap qm;
+    if (!make_tmap_2d(&qm, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Dqk, (uint64_t)a.T * a.H, (uint64_t)a.Dqk * 2,
+                      64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return DSA_ERR_INVALID_ARG;
+    if (a.Dqk == 576 && a.Dv == 512) return run_attn<576, 256>(qm, p, st);
+    if (a.Dqk == 64 && a.Dv == 64) return run_attn<64, 64>(qm, p, st);
+    return DSA_ERR_UNSUPPORTED;
+}
+
+}  // namespace dsa

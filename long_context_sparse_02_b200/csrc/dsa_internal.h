@@ -1,0 +1,97 @@
+// Host-side interfaces between the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "dsa.h"
+
+namespace dsa {
+
+struct DeviceInfo {
+    int device = -1;
+    int sm_count = 0;
+    int max_smem_optin = 0;
+    uint32_t *err = nullptr;  // device address of the error word
+};
+
+// Cached per-device facts for the current device (thread-safe).
+const DeviceInfo *current_device();
+
+// Builds a 2-D tiled tensor map: `inner` elements of `elem_bytes` per row,
+// `outer` rows `row_bytes` apart, box [box_inner, box_outer].
+bool make_tmap_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
+
+// Raises the dynamic shared-memory limit of `fn` once per device.
+bool ensure_smem(const void *fn, int bytes);
+
+struct PagedDev {
+    const int32_t *seq_lens;
+    const int32_t *block_table;
+    int32_t num_seqs, max_blocks, num_pages;
+};
+
+// ---- indexer ---------------------------------------------------------------
+struct IndexerArgs {
+    const uint8_t *q_idx;
+    const float *w;
+    const uint8_t *k_cache;
+    PagedDev pg;
+    const int32_t *q_seq;  // NULL => decode convention
+    const int32_t *q_pos;
+    int32_t T, HI, DI, max_len;
+    float *scores;
+    int64_t ld;
+};
+dsa_status launch_indexer(const IndexerArgs &a, cudaStream_t st);
+
+// ---- top-K ---------------------------------------------------------------------
+enum RowLenMode : int32_t { ROWLEN_ARRAY = 0, ROWLEN_QPOS_PLUS_1 = 1, ROWLEN_SEQ_LENS = 2 };
+struct TopkArgs {
+    const float *scores;
+    int64_t ld;
+    const int32_t *row_len;  // meaning per mode
+    int32_t mode;
+    int32_t R, K, max_row_len;
+    int32_t *idx;
+    void *ws;
+    size_t ws_bytes;
+};
+size_t topk_workspace_bytes(int32_t R, int32_t K, int32_t max_row_len);
+dsa_status launch_topk(const TopkArgs &a, cudaStream_t st);
+
+// ---- gated sparse attention ----------------------------------------------------
+struct AttnArgs {
+    const uint16_t *q;
+    const uint16_t *kv;
+    PagedDev pg;
+    const int32_t *q_seq;  // NULL => query t reads sequence t
+    const int32_t *idx;
+    int32_t K;
+    const uint16_t *gate;
+    float sm_scale;
+    int32_t T, H, Dqk, Dv;
+    uint16_t *out;
+    float *lse;
+    void *ws;
+    size_t ws_bytes;
+};
+size_t attn_workspace_bytes(int32_t T, int32_t H, int32_t K, int32_t Dv);
+dsa_status launch_attn(const AttnArgs &a, cudaStream_t st);
+
+// ---- sliding-window decode -------------------------------------------------------
+struct SwaArgs {
+    const uint16_t *q, *k_ring, *v_ring;
+    const int32_t *seq_lens;
+    int32_t B, H, D, W;
+    float sm_scale;
+    uint16_t *out;
+};
+dsa_status launch_swa(const SwaArgs &a, cudaStream_t st);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace dsa

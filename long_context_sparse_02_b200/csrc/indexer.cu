@@ -1,0 +1,638 @@
+// Stage 1 of the Gated DSA layer: the lightweight FP8 indexer.
+//
+//   I[t,s] = sum_h w[t,h] * ReLU(qI[t,h,:] . kI[s,:])     for s <= q_pos[t]
+//
+// ("Open-Source LLM Architecture Evolution: How Lightweight Sparse Attention
+// Reshapes Long-Context Modeling Efficiency", Architecture Breakdown §2,
+// "Indexer"; "Fine-Grained Sparse Attention in Ultra-Large Parameter Models",
+// §2.2 -- no rotary embedding, so the stored keys are used as they are -- and
+// §2.3 -- heads x 128 dims.)
+//
+// Both kernels put 128 keys on the M side of a tcgen05 e4m3 MMA (two 64-row
+// pages of the paged key cache, fetched by TMA with the 128- or 64-byte
+// swizzle the MMA reads), accumulate in fp32 in tensor memory and apply the
+// ReLU and the w-weighted head reduction in the epilogue warps:
+//   * decode: N = the query's heads (padded to 16); one query per tile; the
+//     tiles of all queries are spread evenly over a persistent grid, so even
+//     one 1M-token query keeps every SM streaming its own slice of keys.
+//   * prefill: N = 256 = a group of 256/HI consecutive queries x HI heads; a
+//     persistent CTA takes whole query groups (snake order, costliest first)
+//     and streams the key tiles of the group's causal range.
+// Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM owner),
+// warps 2..5 = epilogue (one TMEM lane quarter each).
+#include "dsa_device.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+namespace {
+
+struct QInfo {
+    int32_t b;     // sequence
+    int32_t last;  // last history position scored (inclusive); -1 = none
+};
+
+__device__ __forceinline__ QInfo query_info(int t, const int32_t *q_seq, const int32_t *q_pos, const PagedDev &pg,
+                                            int max_len, uint32_t *err) {
+    int b, last;
+    if (q_seq == nullptr) {
+        b = t;
+        if (b >= pg.num_seqs) {
+            record_error(err, DSA_DEVERR_POSITION);
+            return {0, -1};
+        }
+        last = pg.seq_lens[b] - 1;
+    } else {
+        b = q_seq[t];
+        last = q_pos[t];
+        if (b < 0 || b >= pg.num_seqs || last < 0) {
+            record_error(err, DSA_DEVERR_POSITION);
+            return {0, -1};
+        }
+    }
+    const int L = pg.seq_lens[b];
+    if (last >= L) {
+        record_error(err, DSA_DEVERR_POSITION);
+        last = L - 1;
+    }
+    if (last >= max_len) {
+        record_error(err, DSA_DEVERR_SHAPE);
+        last = max_len - 1;
+    }
+    return {b, last};
+}
+
+// Physical page of logical page lp of sequence b, or -1 (recorded) if the
+// table entry is out of range.
+__device__ __forceinline__ int page_of(const PagedDev &pg, int b, int lp, uint32_t *err) {
+    if (lp >= pg.max_blocks) {
+        record_error(err, DSA_DEVERR_PAGE);
+        return -1;
+    }
+    const int p = pg.block_table[(int64_t)b * pg.max_blocks + lp];
+    if (p < 0 || p >= pg.num_pages) {
+        record_error(err, DSA_DEVERR_PAGE);
+        return -1;
+    }
+    return p;
+}
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+constexpr int pow2_cols(int c) { return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512; }
+
+struct IdxParams {
+    const float *w;
+    const int32_t *q_seq, *q_pos;
+    PagedDev pg;
+    int32_t T, HI, max_len;
+    float *scores;
+    int64_t ld;
+    uint32_t *err;
+};
+
+// ============================================================================
+// decode: keys x heads, one query per tile
+// ============================================================================
+
+template <int DI, int NH>
+struct DecCfg {
+    static constexpr int STAGES = DI == 128 ? 8 : 12;
+    static constexpr int ACC = 4;
+    static constexpr int A_BYTES = 128 * DI;
+    static constexpr int B_BYTES = NH * DI;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int TMEM_COLS = pow2_cols(ACC * NH);
+    static constexpr uint32_t SWZ = DI == 128 ? SWZ_128B : SWZ_64B;
+    static constexpr uint32_t SBO = 8 * DI;
+    static constexpr int MAXT = 1024;
+    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * ACC + 1);
+    static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + 4 * (MAXT + 1) + 16;
+    static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+};
+
+// Index t with tstart[t] <= g < tstart[t+1] (tstart non-decreasing, g < tstart[T]).
+__device__ __forceinline__ int locate(const int32_t *tstart, int T, int64_t g) {
+    int lo = 0, hi = T;  // answer in [lo, hi)
+    while (hi - lo > 1) {
+        int mid = (lo + hi) >> 1;
+        if (tstart[mid] <= g) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+template <int DI, int NH>
+__global__ void __launch_bounds__(192, 1)
+    indexer_decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                          const IdxParams p) {
+    using C = DecCfg<DI, NH>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    uint8_t *stages = smem;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::STAGES * C::STAGE_BYTES);
+    uint64_t *empty = full + C::STAGES;
+    uint64_t *tfull = empty + C::STAGES;
+    uint64_t *tempty = tfull + C::ACC;
+    uint64_t *drain = tempty + C::ACC;
+    int32_t *tstart = reinterpret_cast<int32_t *>(drain + 1);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tstart + C::MAXT + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = warp_id(), lane = lane_id();
+    const int T = p.T;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < C::ACC; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        tstart[0] = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&kmap);
+        tma_prefetch_desc(&qmap);
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+    for (int t = threadIdx.x; t < T; t += blockDim.x) {
+        QInfo qi = query_info(t, p.q_seq, p.q_pos, p.pg, p.max_len, nullptr);
+        tstart[t + 1] = (qi.last + 1 + 127) >> 7;
+    }
+    __syncthreads();
+    if (warp == 0) {  // inclusive scan of the per-query tile counts
+        int running = 0;
+        for (int base = 0; base < T; base += 32) {
+            const int i = base + lane;
+            int v = i < T ? tstart[i + 1] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                int n = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += n;
+            }
+            if (i < T) tstart[i + 1] = running + v;
+            running += __shfl_sync(0xffffffffu, v, 31);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int64_t total = tstart[T];
+    const int64_t lo = total * blockIdx.x / gridDim.x;
+    const int64_t hi = total * (blockIdx.x + 1) / gridDim.x;
+    const int n = static_cast<int>(hi - lo);
+
+    if (warp == 0 && lane == 0 && n > 0) {
+        // ---------------- producer ----------------
+        int t = locate(tstart, T, lo);
+        int j = static_cast<int>(lo - tstart[t]);
+        QInfo qi = query_info(t, p.q_seq, p.q_pos, p.pg, p.max_len, p.err);
+        int issued = 0;
+        for (int i = 0; i < n; ++i) {
+            const int s = i % C::STAGES;
+            const uint32_t ph = (i / C::STAGES) & 1;
+            if (!mbar_wait(&empty[s], ph ^ 1, p.err, abort_flag)) break;
+            uint8_t *A = stages + s * C::STAGE_BYTES;
+            uint8_t *B = A + C::A_BYTES;
+            const int pg0 = page_of(p.pg, qi.b, 2 * j, p.err);
+            const int pg1 = (2 * j + 1) * 64 <= qi.last ? page_of(p.pg, qi.b, 2 * j + 1, p.err) : -1;
+            const uint32_t bytes = C::B_BYTES + (pg0 >= 0 ? 64 * DI : 0) + (pg1 >= 0 ? 64 * DI : 0);
+            mbar_expect_tx(&full[s], bytes);
+            if (pg0 >= 0) tma_load_2d(A, &kmap, &full[s], 0, pg0 * 64);
+            if (pg1 >= 0) tma_load_2d(A + 64 * DI, &kmap, &full[s], 0, pg1 * 64);
+            tma_load_2d(B, &qmap, &full[s], 0, t * p.HI);
+            ++issued;
+            if (++j == tstart[t + 1] - tstart[t]) {
+                j = 0;
+                do { ++t; } while (t < T && tstart[t + 1] == tstart[t]);
+                if (t < T) qi = query_info(t, p.q_seq, p.q_pos, p.pg, p.max_len, p.err);
+            }
+        }
+        // never leave a copy in flight behind
+        for (int i = issued - 1; i >= 0 && i >= issued - C::STAGES; --i)
+            mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1, p.err, nullptr);
+    } else if (warp == 1 && lane == 0 && n > 0) {
+        // ---------------- MMA issuer ----------------
+        constexpr uint32_t ID = idesc(0, 0, 0, 0, NH, 128);
+        for (int i = 0; i < n; ++i) {
+            const int s = i % C::STAGES;
+            const uint32_t ph = (i / C::STAGES) & 1;
+            const int a = i % C::ACC;
+            const uint32_t aph = (i / C::ACC) & 1;
+            if (!mbar_wait(&full[s], ph, p.err, abort_flag)) break;
+            if (!mbar_wait(&tempty[a], aph ^ 1, p.err, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t A = smem_u32(stages + s * C::STAGE_BYTES);
+            const uint32_t B = A + C::A_BYTES;
+            const uint32_t d = tmem + a * NH;
+#pragma unroll
+            for (int k = 0; k < DI / 32; ++k)
+                mma_e4m3(d, sdesc(A + 32 * k, 16, C::SBO, C::SWZ), sdesc(B + 32 * k, 16, C::SBO, C::SWZ), ID,
+                         k > 0);
+            mma_commit(&empty[s]);
+            mma_commit(&tfull[a]);
+        }
+        mma_commit(drain);
+        mbar_wait(drain, 0, p.err, nullptr);
+    } else if (warp >= 2 && n > 0) {
+        // ---------------- epilogue ----------------
+        const int q4 = warp & 3;
+        const int row = q4 * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+        int t = locate(tstart, T, lo);
+        int j = static_cast<int>(lo - tstart[t]);
+        QInfo qi = query_info(t, p.q_seq, p.q_pos, p.pg, p.max_len, p.err);
+        float wr[NH];
+#pragma unroll
+        for (int h = 0; h < NH; ++h) wr[h] = h < p.HI ? p.w[(int64_t)t * p.HI + h] : 0.f;
+        for (int i = 0; i < n; ++i) {
+            const int a = i % C::ACC;
+            const uint32_t aph = (i / C::ACC) & 1;
+            if (!mbar_wait(&tfull[a], aph, p.err, abort_flag)) break;
+            tc_fence_after();
+            uint32_t r[NH];
+            const uint32_t ta = tmem + a * NH + lane_off;
+            if constexpr (NH == 16) {
+                tmem_ld16(ta, r);
+            } else {
+#pragma unroll
+                for (int c = 0; c < NH / 32; ++c) tmem_ld32(ta + 32 * c, r + 32 * c);
+            }
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[a]);
+            float sc = 0.f;
+#pragma unroll
+            for (int h = 0; h < NH; ++h)
+                if (h < p.HI) sc = fmaf(wr[h], fmaxf(__uint_as_float(r[h]), 0.f), sc);
+            const int spos = j * 128 + row;
+            if (spos <= qi.last) p.scores[(int64_t)t * p.ld + spos] = sc;
+            if (++j == tstart[t + 1] - tstart[t]) {
+                j = 0;
+                do { ++t; } while (t < T && tstart[t + 1] == tstart[t]);
+                if (t < T) {
+                    qi = query_info(t, p.q_seq, p.q_pos, p.pg, p.max_len, p.err);
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) wr[h] = h < p.HI ? p.w[(int64_t)t * p.HI + h] : 0.f;
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ============================================================================
+// prefill: keys x (query group x heads), N = 256
+// ============================================================================
+
+template <int DI, int HI>
+struct PreCfg {
+    static constexpr int N = 256;
+    static constexpr int G = N / HI;  // queries per group
+    static constexpr int A_BYTES = 128 * DI;
+    static constexpr int B_BYTES = N * DI;
+    static constexpr int ASTAGES = DI == 128 ? 6 : 10;
+    static constexpr int TMEM_COLS = 512;
+    static constexpr uint32_t SWZ = DI == 128 ? SWZ_128B : SWZ_64B;
+    static constexpr uint32_t SBO = 8 * DI;
+    static constexpr int BAR_BYTES = 8 * (2 * ASTAGES + 4 + 4 + 1);
+    static constexpr int TBL = 3 * G;  // three per-role copies of the group table
+    static constexpr int SMEM = 1024 + 2 * B_BYTES + ASTAGES * A_BYTES + BAR_BYTES + 4 * N + 8 * TBL + 16;
+};
+
+// One role's view of a query group: token u's (sequence, last position).
+__device__ __forceinline__ void load_group_tbl(int2 *tbl, int g, int G, const IdxParams &p, bool report, int lane,
+                                               int nthr) {
+    for (int u = lane; u < G; u += nthr) {
+        const int t = g * G + u;
+        int2 v = make_int2(-1, -1);
+        if (t < p.T) {
+            QInfo qi = query_info(t, p.q_seq, p.q_pos, p.pg, p.max_len, report ? p.err : nullptr);
+            v = make_int2(qi.last >= 0 ? qi.b : -1, qi.last);
+        }
+        tbl[u] = v;
+    }
+}
+
+// Next run of consecutive tokens [u, *u1) of one sequence; returns its key
+// tile count.
+__device__ __forceinline__ int next_run(const int2 *tbl, int G, int u, int *u1, int *b) {
+    const int bb = tbl[u].x;
+    int mx = tbl[u].y, v = u + 1;
+    while (v < G && tbl[v].x == bb) {
+        mx = max(mx, tbl[v].y);
+        ++v;
+    }
+    *u1 = v;
+    *b = bb;
+    return bb < 0 ? 0 : (mx + 1 + 127) >> 7;
+}
+
+__device__ __forceinline__ int group_of(int r, int c, int grid, int ngroups) {
+    const int k = r * grid + ((r & 1) ? grid - 1 - c : c);
+    return k < ngroups ? ngroups - 1 - k : -1;
+}
+
+template <int DI, int HI>
+__global__ void __launch_bounds__(192, 1)
+    indexer_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                           const IdxParams p) {
+    using C = PreCfg<DI, HI>;
+    constexpr int G = C::G;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    uint8_t *Bbuf = smem;                     // [2][B_BYTES]
+    uint8_t *Abuf = smem + 2 * C::B_BYTES;    // [ASTAGES][A_BYTES]
+    uint64_t *afull = reinterpret_cast<uint64_t *>(Abuf + C::ASTAGES * C::A_BYTES);
+    uint64_t *aempty = afull + C::ASTAGES;
+    uint64_t *bfull = aempty + C::ASTAGES;
+    uint64_t *bempty = bfull + 2;
+    uint64_t *tfull = bempty + 2;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    float *wbuf = reinterpret_cast<float *>(drain + 1);
+    int2 *tbl_p = reinterpret_cast<int2 *>(wbuf + C::N);
+    int2 *tbl_m = tbl_p + G;
+    int2 *tbl_e = tbl_m + G;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tbl_e + G);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = warp_id(), lane = lane_id();
+    const int ngroups = (p.T + G - 1) / G;
+    const int grid = gridDim.x, cta = blockIdx.x;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::ASTAGES; ++s) {
+            mbar_init(&afull[s], 1);
+            mbar_init(&aempty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bfull[i], 1);
+            mbar_init(&bempty[i], 1);
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&kmap);
+        tma_prefetch_desc(&qmap);
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- producer (warp loads tables, lane 0 issues) ----------------
+        int ac = 0, issued_a = 0, gi = 0;
+        bool ok = true;
+        for (int r = 0; ok; ++r, ++gi) {
+            const int g = group_of(r, cta, grid, ngroups);
+            if (g < 0) break;
+            load_group_tbl(tbl_p, g, G, p, false, lane, 32);
+            __syncwarp();
+            if (lane == 0) {
+                const int bst = gi & 1;
+                if (!mbar_wait(&bempty[bst], ((gi >> 1) & 1) ^ 1, p.err, abort_flag)) ok = false;
+                if (ok) {
+                    mbar_expect_tx(&bfull[bst], C::B_BYTES);
+                    tma_load_2d(Bbuf + bst * C::B_BYTES, &qmap, &bfull[bst], 0, g * G * HI);
+                }
+                for (int u = 0; ok && u < G;) {
+                    int u1, b;
+                    const int nt = next_run(tbl_p, G, u, &u1, &b);
+                    int mx = -1;
+                    for (int v = u; v < u1; ++v) mx = max(mx, tbl_p[v].y);
+                    for (int kt = 0; kt < nt; ++kt) {
+                        const int s = ac % C::ASTAGES;
+                        if (!mbar_wait(&aempty[s], ((ac / C::ASTAGES) & 1) ^ 1, p.err, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t *A = Abuf + s * C::A_BYTES;
+                        const int pg0 = page_of(p.pg, b, 2 * kt, p.err);
+                        const int pg1 = (2 * kt + 1) * 64 <= mx ? page_of(p.pg, b, 2 * kt + 1, p.err) : -1;
+                        const uint32_t bytes = (pg0 >= 0 ? 64 * DI : 0) + (pg1 >= 0 ? 64 * DI : 0);
+                        if (bytes) {
+                            mbar_expect_tx(&afull[s], bytes);
+                            if (pg0 >= 0) tma_load_2d(A, &kmap, &afull[s], 0, pg0 * 64);
+                            if (pg1 >= 0) tma_load_2d(A + 64 * DI, &kmap, &afull[s], 0, pg1 * 64);
+                        } else {
+                            mbar_arrive(&afull[s]);
+                        }
+                        ++ac;
+                        issued_a = ac;
+                    }
+                    u = u1;
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        }
+        if (lane == 0) {
+            for (int i = issued_a - 1; i >= 0 && i >= issued_a - C::ASTAGES; --i)
+                mbar_wait(&afull[i % C::ASTAGES], (i / C::ASTAGES) & 1, p.err, nullptr);
+            if (gi > 0) mbar_wait(&bfull[(gi - 1) & 1], ((gi - 1) >> 1) & 1, p.err, nullptr);
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        constexpr uint32_t ID = idesc(0, 0, 0, 0, C::N, 128);
+        int ac = 0, tc = 0, gi = 0;
+        bool ok = true;
+        for (int r = 0; ok; ++r, ++gi) {
+            const int g = group_of(r, cta, grid, ngroups);
+            if (g < 0) break;
+            load_group_tbl(tbl_m, g, G, p, false, lane, 32);
+            __syncwarp();
+            if (lane == 0) {
+                const int bst = gi & 1;
+                if (!mbar_wait(&bfull[bst], (gi >> 1) & 1, p.err, abort_flag)) ok = false;
+                const uint32_t B = smem_u32(Bbuf + bst * C::B_BYTES);
+                for (int u = 0; ok && u < G;) {
+                    int u1, b;
+                    const int nt = next_run(tbl_m, G, u, &u1, &b);
+                    for (int kt = 0; kt < nt; ++kt) {
+                        const int s = ac % C::ASTAGES;
+                        const int a = tc & 1;
+                        if (!mbar_wait(&afull[s], (ac / C::ASTAGES) & 1, p.err, abort_flag) ||
+                            !mbar_wait(&tempty[a], ((tc >> 1) & 1) ^ 1, p.err, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t A = smem_u32(Abuf + s * C::A_BYTES);
+#pragma unroll
+                        for (int k = 0; k < DI / 32; ++k)
+                            mma_e4m3(tmem + a * C::N, sdesc(A + 32 * k, 16, C::SBO, C::SWZ),
+                                     sdesc(B + 32 * k, 16, C::SBO, C::SWZ), ID, k > 0);
+                        mma_commit(&aempty[s]);
+                        mma_commit(&tfull[a]);
+                        ++ac;
+                        ++tc;
+                    }
+                    u = u1;
+                }
+                if (ok) mma_commit(&bempty[bst]);
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        }
+        if (lane == 0) {
+            mma_commit(drain);
+            mbar_wait(drain, 0, p.err, nullptr);
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5) ----------------
+        const int et = threadIdx.x - 64;  // 0..127
+        const int q4 = warp & 3;
+        const int row = q4 * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+        int tc = 0;
+        bool ok = true;
+        for (int r = 0; ok; ++r) {
+            const int g = group_of(r, cta, grid, ngroups);
+            if (g < 0) break;
+            named_bar_sync(1, 128);
+            load_group_tbl(tbl_e, g, G, p, true, et, 128);
+            for (int i = et; i < C::N; i += 128) {
+                const int t = g * G + i / HI;
+                wbuf[i] = t < p.T ? p.w[(int64_t)t * HI + (i % HI)] : 0.f;
+            }
+            named_bar_sync(1, 128);
+            for (int u = 0; ok && u < G;) {
+                int u1, b;
+                const int nt = next_run(tbl_e, G, u, &u1, &b);
+                for (int kt = 0; kt < nt; ++kt) {
+                    const int a = tc & 1;
+                    if (!mbar_wait(&tfull[a], (tc >> 1) & 1, p.err, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int spos = kt * 128 + row;
+                    const uint32_t ta = tmem + a * C::N + lane_off;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int cc = 0; cc < C::N / 32; ++cc) {
+                        uint32_t rr[32];
+                        tmem_ld32(ta + 32 * cc, rr);
+                        tmem_wait_ld();
+                        if constexpr (HI >= 32) {
+                            const int tok = (cc * 32) / HI;
+                            const int h0 = (cc * 32) % HI;
+#pragma unroll
+                            for (int h = 0; h < 32; ++h)
+                                acc = fmaf(wbuf[tok * HI + h0 + h], fmaxf(__uint_as_float(rr[h]), 0.f), acc);
+                            if (h0 + 32 == HI) {
+                                const int2 info = tbl_e[tok];
+                                if (tok >= u && tok < u1 && spos <= info.y)
+                                    p.scores[(int64_t)(g * G + tok) * p.ld + spos] = acc;
+                                acc = 0.f;
+                            }
+                        } else {
+#pragma unroll
+                            for (int uu = 0; uu < 32 / HI; ++uu) {
+                                const int tok = (cc * 32) / HI + uu;
+                                float sc = 0.f;
+#pragma unroll
+                                for (int h = 0; h < HI; ++h)
+                                    sc = fmaf(wbuf[tok * HI + h], fmaxf(__uint_as_float(rr[uu * HI + h]), 0.f), sc);
+                                const int2 info = tbl_e[tok];
+                                if (tok >= u && tok < u1 && spos <= info.y)
+                                    p.scores[(int64_t)(g * G + tok) * p.ld + spos] = sc;
+                            }
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[a]);
+                    ++tc;
+                }
+                u = u1;
+            }
+            ok = !*abort_flag;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+template <int DI, int NH>
+dsa_status run_decode(const CUtensorMap &km, const CUtensorMap &qm, const IdxParams &p, int grid, cudaStream_t st) {
+    using C = DecCfg<DI, NH>;
+    auto fn = indexer_decode_kernel<DI, NH>;
+    if (!ensure_smem(reinterpret_cast<const void *>(fn), C::SMEM)) return DSA_ERR_CUDA;
+    fn<<<grid, 192, C::SMEM, st>>>(km, qm, p);
+    return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+template <int DI, int HI>
+dsa_status run_prefill(const CUtensorMap &km, const CUtensorMap &qm, const IdxParams &p, int grid,
+                       cudaStream_t st) {
+    using C = PreCfg<DI, HI>;
+    auto fn = indexer_prefill_kernel<DI, HI>;
+    if (!ensure_smem(reinterpret_cast<const void *>(fn), C::SMEM)) return DSA_ERR_CUDA;
+    fn<<<grid, 192, C::SMEM, st>>>(km, qm, p);
+    return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+}  // namespace
+
+dsa_status launch_indexer(const IndexerArgs &a, cudaStream_t st) {
+    const DeviceInfo *dev = current_device();
+    if (!dev) return DSA_ERR_CUDA;
+    if (a.T == 0) return DSA_OK;
+    IdxParams p{a.w, a.q_seq, a.q_pos, a.pg, a.T, a.HI, a.max_len, a.scores, a.ld, dev->err};
+    const CUtensorMapSwizzle swz = a.DI == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    CUtensorMap km, qm;
+    if (!make_tmap_2d(&km, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.DI, (uint64_t)a.pg.num_pages * 64, a.DI,
+                      a.DI, 64, swz))
+        return DSA_ERR_INVALID_ARG;
+    const bool decode = a.q_seq == nullptr || a.T <= 64;
+    if (decode) {
+        if (a.T > DecCfg<128, 32>::MAXT) return DSA_ERR_UNSUPPORTED;
+        const int NH = a.HI <= 16 ? 16 : a.HI <= 32 ? 32 : 64;
+        if (!make_tmap_2d(&qm, a.q_idx, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.DI, (uint64_t)a.T * a.HI, a.DI, a.DI, NH,
+                          swz))
+            return DSA_ERR_INVALID_ARG;
+        const int64_t tiles_bound = (int64_t)a.T * ((a.max_len + 127) / 128);
+        const int grid = (int)(tiles_bound < dev->sm_count ? tiles_bound : dev->sm_count);
+        if (grid <= 0) return DSA_OK;
+        if (a.DI == 128) {
+            if (NH == 16) return run_decode<128, 16>(km, qm, p, grid, st);
+            if (NH == 32) return run_decode<128, 32>(km, qm, p, grid, st);
+            return run_decode<128, 64>(km, qm, p, grid, st);
+        }
+        if (NH == 16) return run_decode<64, 16>(km, qm, p, grid, st);
+        if (NH == 32) return run_decode<64, 32>(km, qm, p, grid, st);
+        return run_decode<64, 64>(km, qm, p, grid, st);
+    }
+    if (!make_tmap_2d(&qm, a.q_idx, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.DI, (uint64_t)a.T * a.HI, a.DI, a.DI, 256, swz))
+        return DSA_ERR_INVALID_ARG;
+    const int G = 256 / a.HI;
+    const int ngroups = (a.T + G - 1) / G;
+    const int grid = ngroups < dev->sm_count ? ngroups : dev->sm_count;
+#define DSA_PRE(DIV, HIV) \
+    if (a.DI == DIV && a.HI == HIV) return run_prefill<DIV, HIV>(km, qm, p, grid, st);
+    DSA_PRE(128, 4) DSA_PRE(128, 8) DSA_PRE(128, 16) DSA_PRE(128, 32) DSA_PRE(128, 64)
+    DSA_PRE(64, 4) DSA_PRE(64, 8) DSA_PRE(64, 16) DSA_PRE(64, 32) DSA_PRE(64, 64)
+#undef DSA_PRE
+    return DSA_ERR_UNSUPPORTED;
+}
+
+}  // namespace dsa

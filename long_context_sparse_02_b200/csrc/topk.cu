@@ -1,0 +1,361 @@
+// Stage 2 of the Gated DSA layer: per-row top-K selection.
+//
+// Keeps the K highest indexer scores of each row ("Open-Source LLM
+// Architecture Evolution", Architecture Breakdown §2, "Top-K selection",
+// K = 2048; "Fine-Grained Sparse Attention in Ultra-Large Parameter Models",
+// §2.1), every position when the row is not longer than K.  Ties go to the
+// lower position and -0.0 equals +0.0.  The kept positions are written in
+// ascending order, padded with -1.
+//
+// Exact radix select on order-preserving 32-bit keys: three digit passes
+// (11, 11 and 10 bits) find the K-th largest key tau and the number `need`
+// of keys equal to tau that are kept; a stable compaction in position order
+// then takes every key > tau and the first `need` keys == tau.
+//   * rows up to SMALL_CAP keys: one CTA per row, keys resident in shared
+//     memory, histograms in shared memory;
+//   * longer rows: CHUNK-key slices per CTA, per-row global histograms, the
+//     last CTA of a pass (atomic ticket, no waiting) picks the digit; then a
+//     count pass and an offset-and-write pass.
+#include "dsa_device.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+namespace {
+
+constexpr int SMALL_THREADS = 1024;
+constexpr int SMALL_CAP = 49152;  // keys resident in shared memory (192 KB)
+constexpr int CHUNK = 4096;       // keys per CTA on the multi-CTA path
+constexpr int MULTI_THREADS = 256;
+constexpr int HBINS = 2048;
+
+struct Pass {
+    int shift, bits;
+};
+__device__ __constant__ Pass kPass[3] = {{21, 11}, {10, 11}, {0, 10}};
+
+__device__ __forceinline__ int row_length(const TopkArgs &a, int r, uint32_t *err) {
+    int n;
+    if (a.mode == ROWLEN_ARRAY) n = a.row_len[r];
+    else if (a.mode == ROWLEN_QPOS_PLUS_1) n = a.row_len[r] + 1;
+    else n = a.row_len[r];  // ROWLEN_SEQ_LENS: decode, row r = sequence r
+    if (n < 0) {
+        record_error(err, DSA_DEVERR_SHAPE);
+        n = 0;
+    }
+    if (n > a.max_row_len) {
+        record_error(err, DSA_DEVERR_SHAPE);
+        n = a.max_row_len;
+    }
+    return n;
+}
+
+// Picks, from a histogram of `nb` bins, the bin b holding the remaining-th
+// largest key: sum(hist[b+1:]) < remaining <= sum(hist[b:]).  Block-wide;
+// returns (b, keys in bins above b) in *out (shared).
+template <int NT>
+__device__ void pick_bin(const uint32_t *hist, int nb, uint32_t remaining, uint32_t *scan, int2 *out) {
+    const int tid = threadIdx.x;
+    constexpr int PER = HBINS / NT > 0 ? HBINS / NT : 1;
+    // thread tid owns bins [tid*PER, tid*PER+PER) counted from the TOP
+    uint32_t local = 0;
+    for (int i = 0; i < PER; ++i) {
+        const int bin = nb - 1 - (tid * PER + i);
+        if (bin >= 0) local += hist[bin];
+    }
+    scan[tid] = local;
+    __syncthreads();
+    // inclusive scan over threads (Hillis-Steele)
+    for (int o = 1; o < NT; o <<= 1) {
+        uint32_t v = tid >= o ? scan[tid - o] : 0;
+        __syncthreads();
+        scan[tid] += v;
+        __syncthreads();
+    }
+    const uint32_t incl = scan[tid];
+    const uint32_t excl = incl - local;
+    if (excl < remaining && remaining <= incl) {
+        uint32_t above = excl;
+        for (int i = 0; i < PER; ++i) {
+            const int bin = nb - 1 - (tid * PER + i);
+            if (bin < 0) break;
+            if (above + hist[bin] >= remaining) {
+                *out = make_int2(bin, (int)above);
+                break;
+            }
+            above += hist[bin];
+        }
+    }
+    __syncthreads();
+}
+
+// Block-wide exclusive scan of two small counters packed as (hi16, lo16).
+template <int NT>
+__device__ __forceinline__ uint32_t block_excl_scan_packed(uint32_t v, uint32_t *wsum, uint32_t *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        uint32_t n = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += n;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t s = lane < NT / 32 ? wsum[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            uint32_t n = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += n;
+        }
+        if (lane < NT / 32) wsum[lane] = s;
+        if (lane == 31) *total = s;
+    }
+    __syncthreads();
+    const uint32_t base = warp > 0 ? wsum[warp - 1] : 0;
+    const uint32_t res = base + x - v;
+    __syncthreads();
+    return res;
+}
+
+// Writes the kept positions of [s0, s1) in order.  gt_before/eq_before count
+// keys > tau / == tau before s0 in the row.
+template <int NT, typename KeyAt>
+__device__ void compact(KeyAt key_at, int s0, int s1, uint32_t tau, uint32_t need, uint32_t gt_before,
+                        uint32_t eq_before, int32_t *out, int K, uint32_t *wsum, uint32_t *total, uint32_t *err) {
+    for (int base = s0; base < s1; base += NT) {
+        const int s = base + threadIdx.x;
+        uint32_t gt = 0, eq = 0;
+        if (s < s1) {
+            const uint32_t k = key_at(s);
+            gt = k > tau;
+            eq = k == tau;
+        }
+        const uint32_t pk = block_excl_scan_packed<NT>((gt << 16) | eq, wsum, total);
+        const uint32_t tot = *total;
+        const uint32_t e_before = eq_before + (pk & 0xFFFFu);
+        const uint32_t g_before = gt_before + (pk >> 16);
+        if (gt || (eq && e_before < need)) {
+            const uint32_t slot = g_before + min(e_before, need);
+            if (slot < (uint32_t)K) out[slot] = s;
+            else record_error(err, DSA_DEVERR_SHAPE);
+        }
+        gt_before += tot >> 16;
+        eq_before += tot & 0xFFFFu;
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// one CTA per row, keys in shared memory
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(SMALL_THREADS, 1) topk_small_kernel(const TopkArgs a, uint32_t *err) {
+    extern __shared__ uint32_t sm[];
+    uint32_t *hist = sm;                   // [HBINS]
+    uint32_t *scan = hist + HBINS;         // [SMALL_THREADS]
+    uint32_t *wsum = scan + SMALL_THREADS;  // [32]
+    uint32_t *misc = wsum + 32;            // [8]
+    uint32_t *keys = misc + 8;             // [max_row_len]
+    const int r = blockIdx.x;
+    const int n = row_length(a, r, err);
+    int32_t *out = a.idx + (int64_t)r * a.K;
+    if (n <= a.K) {
+        for (int j = threadIdx.x; j < a.K; j += SMALL_THREADS) out[j] = j < n ? j : -1;
+        return;
+    }
+    const float *row = a.scores + (int64_t)r * a.ld;
+    for (int s = threadIdx.x; s < n; s += SMALL_THREADS) keys[s] = score_key(row[s]);
+    uint32_t prefix = 0, remaining = (uint32_t)a.K;
+    for (int ps = 0; ps < 3; ++ps) {
+        const int shift = kPass[ps].shift, bits = kPass[ps].bits;
+        const int nb = 1 << bits;
+        for (int i = threadIdx.x; i < nb; i += SMALL_THREADS) hist[i] = 0;
+        __syncthreads();
+        const int hs = shift + bits;
+        for (int s = threadIdx.x; s < n; s += SMALL_THREADS) {
+            const uint32_t k = keys[s];
+            if (hs == 32 || (k >> hs) == prefix) atomicAdd(&hist[(k >> shift) & (nb - 1)], 1u);
+        }
+        __syncthreads();
+        int2 *res = reinterpret_cast<int2 *>(misc);
+        if (threadIdx.x == 0) *res = make_int2(0, 0);
+        __syncthreads();
+        pick_bin<SMALL_THREADS>(hist, nb, remaining, scan, res);
+        prefix = (prefix << bits) | (uint32_t)res->x;
+        remaining -= (uint32_t)res->y;
+        __syncthreads();
+    }
+    compact<SMALL_THREADS>([&](int s) { return keys[s]; }, 0, n, prefix, remaining, 0, 0, out, a.K, wsum, misc + 4,
+                          err);
+}
+
+// ---------------------------------------------------------------------------
+// long rows: several CTAs per row
+// ---------------------------------------------------------------------------
+struct RowState {
+    uint32_t prefix, remaining;
+    uint32_t ticket[3];
+    uint32_t pad[3];
+};
+
+struct MultiWs {
+    uint32_t *hist;    // [R][3][HBINS]
+    RowState *state;   // [R]
+    uint32_t *counts;  // [R][nchunks][2]
+    int nchunks;
+};
+
+__host__ __device__ inline MultiWs carve_multi(void *ws, int R, int max_row_len) {
+    MultiWs m;
+    uint8_t *p = static_cast<uint8_t *>(ws);
+    m.hist = reinterpret_cast<uint32_t *>(p);
+    p += (size_t)R * 3 * HBINS * 4;
+    m.state = reinterpret_cast<RowState *>(p);
+    p += (size_t)R * sizeof(RowState);
+    m.counts = reinterpret_cast<uint32_t *>(p);
+    m.nchunks = (max_row_len + CHUNK - 1) / CHUNK;
+    return m;
+}
+__host__ inline size_t multi_zero_bytes(int R) { return (size_t)R * (3 * HBINS * 4 + sizeof(RowState)); }
+
+__device__ __forceinline__ uint32_t key_at_global(const float *row, int s) { return score_key(__ldg(row + s)); }
+
+__global__ void __launch_bounds__(MULTI_THREADS) topk_pass_kernel(const TopkArgs a, MultiWs m, int ps,
+                                                                 uint32_t *err) {
+    __shared__ uint32_t hist[HBINS];
+    __shared__ uint32_t scan[MULTI_THREADS];
+    __shared__ int2 res;
+    __shared__ uint32_t is_last;
+    const int r = blockIdx.y, c = blockIdx.x;
+    const int n = row_length(a, r, ps == 0 ? err : nullptr);
+    if (n <= a.K) return;
+    const int nch = (n + CHUNK - 1) / CHUNK;
+    if (c >= nch) return;
+    RowState *st = m.state + r;
+    const uint32_t prefix = ps == 0 ? 0u : st->prefix;
+    const uint32_t remaining = ps == 0 ? (uint32_t)a.K : st->remaining;
+    const int shift = kPass[ps].shift, bits = kPass[ps].bits, nb = 1 << bits, hs = shift + bits;
+    for (int i = threadIdx.x; i < nb; i += MULTI_THREADS) hist[i] = 0;
+    __syncthreads();
+    const float *row = a.scores + (int64_t)r * a.ld;
+    const int s1 = min(n, (c + 1) * CHUNK);
+    for (int s = c * CHUNK + threadIdx.x; s < s1; s += MULTI_THREADS) {
+        const uint32_t k = key_at_global(row, s);
+        if (hs == 32 || (k >> hs) == prefix) atomicAdd(&hist[(k >> shift) & (nb - 1)], 1u);
+    }
+    __syncthreads();
+    uint32_t *gh = m.hist + ((size_t)r * 3 + ps) * HBINS;
+    for (int i = threadIdx.x; i < nb; i += MULTI_THREADS)
+        if (hist[i]) atomicAdd(&gh[i], hist[i]);
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = atomicAdd(&st->ticket[ps], 1u) == (uint32_t)(nch - 1);
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    for (int i = threadIdx.x; i < nb; i += MULTI_THREADS) hist[i] = __ldcg(&gh[i]);
+    __syncthreads();
+    pick_bin<MULTI_THREADS>(hist, nb, remaining, scan, &res);
+    if (threadIdx.x == 0) {
+        st->prefix = (prefix << bits) | (uint32_t)res.x;
+        st->remaining = remaining - (uint32_t)res.y;
+    }
+}
+
+__global__ void __launch_bounds__(MULTI_THREADS) topk_count_kernel(const TopkArgs a, MultiWs m) {
+    __shared__ uint32_t wsum[32];
+    const int r = blockIdx.y, c = blockIdx.x;
+    const int n = row_length(a, r, nullptr);
+    if (n <= a.K) return;
+    const int nch = (n + CHUNK - 1) / CHUNK;
+    if (c >= nch) return;
+    const uint32_t tau = m.state[r].prefix;
+    const float *row = a.scores + (int64_t)r * a.ld;
+    const int s1 = min(n, (c + 1) * CHUNK);
+    uint32_t gt = 0, eq = 0;
+    for (int s = c * CHUNK + threadIdx.x; s < s1; s += MULTI_THREADS) {
+        const uint32_t k = key_at_global(row, s);
+        gt += k > tau;
+        eq += k == tau;
+    }
+    uint32_t v = (gt << 16) | eq;  // <= CHUNK each: fits in 16 bits
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) wsum[warp] = v;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t t = 0;
+        for (int w = 0; w < MULTI_THREADS / 32; ++w) t += wsum[w];
+        m.counts[((size_t)r * m.nchunks + c) * 2 + 0] = t >> 16;
+        m.counts[((size_t)r * m.nchunks + c) * 2 + 1] = t & 0xFFFFu;
+    }
+}
+
+__global__ void __launch_bounds__(MULTI_THREADS) topk_write_kernel(const TopkArgs a, MultiWs m, uint32_t *err) {
+    __shared__ uint32_t wsum[32];
+    __shared__ uint32_t tot[2];
+    __shared__ uint32_t before[2];
+    const int r = blockIdx.y, c = blockIdx.x;
+    const int n = row_length(a, r, nullptr);
+    int32_t *out = a.idx + (int64_t)r * a.K;
+    if (n <= a.K) {
+        for (int j = c * CHUNK + threadIdx.x; j < min(a.K, (c + 1) * CHUNK); j += MULTI_THREADS)
+            out[j] = j < n ? j : -1;
+        return;
+    }
+    const int nch = (n + CHUNK - 1) / CHUNK;
+    if (c >= nch) return;
+    const uint32_t tau = m.state[r].prefix, need = m.state[r].remaining;
+    if (threadIdx.x < 32) {
+        uint32_t g = 0, e = 0;
+        for (int i = threadIdx.x; i < c; i += 32) {
+            g += m.counts[((size_t)r * m.nchunks + i) * 2 + 0];
+            e += m.counts[((size_t)r * m.nchunks + i) * 2 + 1];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            g += __shfl_xor_sync(0xffffffffu, g, o);
+            e += __shfl_xor_sync(0xffffffffu, e, o);
+        }
+        if (threadIdx.x == 0) {
+            before[0] = g;
+            before[1] = e;
+        }
+    }
+    __syncthreads();
+    const float *row = a.scores + (int64_t)r * a.ld;
+    compact<MULTI_THREADS>([&](int s) { return key_at_global(row, s); }, c * CHUNK, min(n, (c + 1) * CHUNK), tau,
+                           need, before[0], before[1], out, a.K, wsum, tot, err);
+}
+
+}  // namespace
+
+size_t topk_workspace_bytes(int32_t R, int32_t K, int32_t max_row_len) {
+    (void)K;
+    if (max_row_len <= SMALL_CAP) return 0;
+    const int nch = (max_row_len + CHUNK - 1) / CHUNK;
+    return align_up(multi_zero_bytes(R) + (size_t)R * nch * 2 * 4, 256);
+}
+
+dsa_status launch_topk(const TopkArgs &a, cudaStream_t st) {
+    const DeviceInfo *dev = current_device();
+    if (!dev) return DSA_ERR_CUDA;
+    if (a.R == 0) return DSA_OK;
+    if (a.max_row_len <= SMALL_CAP) {
+        const int smem = (HBINS + SMALL_THREADS + 32 + 8) * 4 + a.max_row_len * 4;
+        if (!ensure_smem(reinterpret_cast<const void *>(topk_small_kernel), smem)) return DSA_ERR_CUDA;
+        topk_small_kernel<<<a.R, SMALL_THREADS, smem, st>>>(a, dev->err);
+        return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+    }
+    const size_t need = topk_workspace_bytes(a.R, a.K, a.max_row_len);
+    if (a.ws == nullptr || a.ws_bytes < need) return DSA_ERR_WORKSPACE;
+    MultiWs m = carve_multi(a.ws, a.R, a.max_row_len);
+    if (cudaMemsetAsync(a.ws, 0, multi_zero_bytes(a.R), st) != cudaSuccess) return DSA_ERR_CUDA;
+    dim3 grid(m.nchunks, a.R);
+    for (int ps = 0; ps < 3; ++ps) topk_pass_kernel<<<grid, MULTI_THREADS, 0, st>>>(a, m, ps, dev->err);
+    topk_count_kernel<<<grid, MULTI_THREADS, 0, st>>>(a, m);
+    topk_write_kernel<<<grid, MULTI_THREADS, 0, st>>>(a, m, dev->err);
+    return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+}  // namespace dsa

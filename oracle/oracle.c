@@ -21,8 +21,9 @@
  *        and DSA hybrid, 16-head indexer, top 2,048, FP8).
  *
  * Every function returns 0 on success and a negative code on bad input.
- * Loops run over queries in parallel with OpenMP; each query's arithmetic is
- * sequential and in the order written.
+ * OpenMP spreads independent outputs (key positions, heads, rows) over the
+ * host's cores; every output's own arithmetic is sequential, in the order
+ * written, so results do not depend on the thread count.
  */
 #include <math.h>
 #include <stdint.h>
@@ -94,18 +95,18 @@ int orc_indexer_scores(const uint8_t *q_idx, const float *w,
                        float *scores, int64_t ld)
 {
     int bad = 0;
-#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    double *q = (double *)malloc(sizeof(double) * (size_t)HI * DI);
     for (int t = 0; t < T; ++t) {
         int b = q_seq[t];
         int64_t p = q_pos[t];
         if (b < 0 || b >= num_seqs || p < 0 || p >= seq_lens[b] || p >= ld) { bad |= 1; continue; }
-        double *q = (double *)malloc(sizeof(double) * (size_t)HI * DI);
         for (int i = 0; i < HI * DI; ++i)
             q[i] = orc_e4m3_to_f64(q_idx[(int64_t)t * HI * DI + i]);
+#pragma omp parallel for schedule(static) reduction(| : bad)
         for (int64_t s = 0; s <= p; ++s) {
             int64_t r = orc_row_index(seq_lens, block_table, num_seqs, max_blocks,
                                       page_size, num_pages, b, s);
-            if (r < 0) { bad |= 1; break; }
+            if (r < 0) { bad |= 1; continue; }
             const uint8_t *k = k_cache + r * DI;
             double I = 0.0;
             for (int h = 0; h < HI; ++h) {
@@ -117,8 +118,8 @@ int orc_indexer_scores(const uint8_t *q_idx, const float *w,
             }
             scores[t * ld + s] = (float)I;
         }
-        free(q);
     }
+    free(q);
     return bad ? ORC_EBAD : 0;
 }
 
@@ -198,12 +199,9 @@ int orc_sparse_attn(const uint16_t *q, const uint16_t *kv_cache,
 {
     int bad = 0;
     if (Dv > Dqk) return ORC_EBAD;
-#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (size_t)(K > 0 ? K : 1));
     for (int t = 0; t < T; ++t) {
         int b = q_seq[t];
-        int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (size_t)K);
-        double *lg = (double *)malloc(sizeof(double) * (size_t)K);
-        double *qv = (double *)malloc(sizeof(double) * (size_t)Dqk);
         int n = 0;
         for (int j = 0; j < K; ++j) {
             int32_t pos = idx[(int64_t)t * K + j];
@@ -213,15 +211,18 @@ int orc_sparse_attn(const uint16_t *q, const uint16_t *kv_cache,
             if (r < 0) { bad |= 1; continue; }
             rows[n++] = r;
         }
+#pragma omp parallel for schedule(dynamic, 1)
         for (int h = 0; h < H; ++h) {
             const uint16_t *qh = q + ((int64_t)t * H + h) * Dqk;
             double *o = out + ((int64_t)t * H + h) * Dv;
-            for (int d = 0; d < Dqk; ++d) qv[d] = orc_bf16_to_f64(qh[d]);
             if (n == 0) {
                 for (int d = 0; d < Dv; ++d) o[d] = 0.0;
                 if (lse) lse[(int64_t)t * H + h] = -INFINITY;
                 continue;
             }
+            double *qv = (double *)malloc(sizeof(double) * (size_t)Dqk);
+            double *lg = (double *)malloc(sizeof(double) * (size_t)n);
+            for (int d = 0; d < Dqk; ++d) qv[d] = orc_bf16_to_f64(qh[d]);
             double m = -INFINITY;
             for (int j = 0; j < n; ++j) {
                 const uint16_t *c = kv_cache + rows[j] * Dqk;
@@ -242,9 +243,10 @@ int orc_sparse_attn(const uint16_t *q, const uint16_t *kv_cache,
             double sig = 1.0 / (1.0 + exp(-g));
             for (int d = 0; d < Dv; ++d) o[d] *= sig;
             if (lse) lse[(int64_t)t * H + h] = m + log(Z);
+            free(qv); free(lg);
         }
-        free(rows); free(lg); free(qv);
     }
+    free(rows);
     return bad ? ORC_EBAD : 0;
 }
 
@@ -261,14 +263,16 @@ int orc_swa_decode(const uint16_t *q, const uint16_t *k_ring,
                    int H, int D, int W, double sm_scale, double *out)
 {
     int bad = 0;
-#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int b = 0; b < B; ++b)
+        if (seq_lens[b] <= 0) bad |= 1;
+    if (bad) return ORC_EBAD;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
     for (int b = 0; b < B; ++b) {
-        int64_t L = seq_lens[b];
-        if (L <= 0) { bad |= 1; continue; }
-        int64_t p0 = L - W > 0 ? L - W : 0;
-        int n = (int)(L - p0);
-        double *lg = (double *)malloc(sizeof(double) * (size_t)n);
         for (int h = 0; h < H; ++h) {
+            int64_t L = seq_lens[b];
+            int64_t p0 = L - W > 0 ? L - W : 0;
+            int n = (int)(L - p0);
+            double *lg = (double *)malloc(sizeof(double) * (size_t)n);
             const uint16_t *qh = q + ((int64_t)b * H + h) * D;
             double m = -INFINITY;
             for (int i = 0; i < n; ++i) {
@@ -289,10 +293,10 @@ int orc_swa_decode(const uint16_t *q, const uint16_t *k_ring,
                 const uint16_t *v = v_ring + (((int64_t)b * W + slot) * H + h) * D;
                 for (int d = 0; d < D; ++d) o[d] += lg[i] / Z * orc_bf16_to_f64(v[d]);
             }
+            free(lg);
         }
-        free(lg);
     }
-    return bad ? ORC_EBAD : 0;
+    return 0;
 }
 
 /* ---- the layer: the three stages in order ---------------------------------- */
