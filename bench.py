@@ -1,0 +1,499 @@
+#!/usr/bin/env python3
+"""Gated DSA layer benchmark on B200.
+
+Headline (one JSON line): decode tokens/s of one Gated DSA layer at a 128K
+context, batch 8 -- 32x128 e4m3 indexer without RoPE, top-K = 2048, 128
+query heads over the 576-wide paged latent cache (512 value dims), sigmoid
+gate -- measured through the C ABI (dsa_layer_forward) on synthetic inputs
+already resident in HBM.  Also reported: the dominant kernel (the decode
+indexer's key stream) against the measured HBM copy bandwidth, the per-stage
+split, the prefill indexer (T = 32768, 16x128) against a measured FP8 GEMM
+peak, an end-to-end figure through host buffers, the CPU oracle on the
+host's cores, and the SM clocks seen during the timed region.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Under torchrun (N > 1) every rank serves its own batch of 8 sequences (the
+path shards by sequence; no collective on the data path): weak scaling,
+value = tokens of all ranks / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "DSA-layer decode tokens/s @128K ctx; prefill indexer TFLOPS & % HBM/FP8 roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20   # > 126 MB L2
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "indexer_decode_B8_L131072.md")
+
+
+# ---------------------------------------------------------------- helpers
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=8)
+    ap.add_argument("--context", type=int, default=131072)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the prefill-indexer, e2e, CPU-baseline and parity legs (profiling runs)")
+    ap.add_argument("--ref-budget-s", type=float, default=120.0,
+                    help="wall-clock budget of the --impl reference run")
+    return ap.parse_args(argv)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured (MEASURED_PEAKS.json)"
+    return dict(FALLBACK_PEAKS), "fallback (no MEASURED_PEAKS.json)"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def aggregate(local_ms: float, local_tokens: int, world: int):
+    """Max-over-ranks time and summed tokens (collective only when world > 1)."""
+    if world == 1:
+        return local_ms, local_tokens
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([local_ms], dtype=torch.float64, device=dev)
+    n = torch.tensor([float(local_tokens)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return float(t.item()), int(n.item())
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+    BAD = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+    def __init__(self, torch_device: int, period_s: float = 0.002):
+        self.samples = []
+        self.period = period_s
+        self.ok = False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(torch_device).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = repr(e)
+
+    def _reasons(self):
+        nv = self.nv
+        f = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return int(f(self.h))
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append((self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM), self._reasons()))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+        return False
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": getattr(self, "err", "no NVML")}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        names = [n for b, n in self.REASONS.items() if bits & b]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+    def rejected(self):
+        s = self.summary()
+        return bool(set(s.get("reasons", [])) & self.BAD)
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(ROOT, "long_context_sparse_02_b200", "csrc", n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """dram read+write bytes per launch of the decode indexer from the committed
+    ncu summary, or None when the kernel source changed since that capture."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None, "no ncu summary"
+    txt = open(PROFILE_SUMMARY).read()
+    m = re.search(r"source_sha256_16:\s*([0-9a-f]{16})", txt)
+    t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not m or not t:
+        return None, "summary lacks traffic/source hash"
+    if m.group(1) != source_hash("indexer.cu", "dsa_device.cuh"):
+        return None, "indexer source changed since the ncu capture"
+    return float(t.group(1)), "ncu capture (profiles/)"
+
+
+# ---------------------------------------------------------------- algorithmic work
+
+def decode_bytes(case):
+    """Bytes the decode layer must move (no score round trip), and the indexer
+    kernel's own I/O (its key stream, queries, weights and the scores it writes)."""
+    L = case.seq_lens.astype(float)
+    kI = float((L * case.DI).sum())
+    qI = case.T * case.HI * case.DI + case.T * case.HI * 4
+    rows = float(sum(min(case.K, int(x)) for x in case.seq_lens))
+    gather = rows * case.Dqk * 2
+    q = case.T * case.H * case.Dqk * 2
+    gate = case.T * case.H * 2
+    out = case.T * case.H * case.Dv * 2
+    layer = kI + qI + gather + q + gate + out
+    indexer = kI + qI + float(L.sum()) * 4
+    return layer, indexer
+
+
+# ---------------------------------------------------------------- native arm
+
+def run_native(args):
+    import numpy as np
+    import torch
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+    from long_context_sparse_02_b200 import build, synth
+    build.build()
+    from long_context_sparse_02_b200 import _lib
+    from long_context_sparse_02_b200.runtime import LayerOnDevice, to_dev
+
+    B, Lctx = args.batch, args.context
+    case = synth.decode_case(args.seed + 1000 * rank, [Lctx] * B, HI=32, name=f"decode_B{B}_L{Lctx}")
+    lay = LayerOnDevice(case, decode=True, want_idx=True)
+    launches = _lib.layer_kernel_launches(lay.args)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    _lib.device_error(reset=True)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        lay.forward()
+    barrier()
+
+    # ---- timed region: K steps of dsa_layer_forward, L2 flushed between steps
+    def timed(fn, K):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        barrier()
+        for s, e in ev:
+            flush.zero_()
+            s.record(stream)
+            fn()
+            e.record(stream)
+        barrier()
+        return [s.elapsed_time(e) for s, e in ev]
+
+    for attempt in range(2):
+        clk = ClockSampler(local)
+        with clk:
+            step_ms = timed(lay.forward, args.steps)
+        if not clk.rejected():
+            break
+    total_ms = sum(step_ms)
+    err = _lib.device_error(reset=True)
+    if err:
+        raise RuntimeError(f"device error word {err:#x} after the timed region")
+    max_ms, tokens = aggregate(total_ms, B * args.steps, world)
+    value = tokens / (max_ms / 1e3)
+
+    # ---- per-stage split (the same kernels, one entry point each)
+    ld = (lay.max_len + 3) // 4 * 4
+    scores = torch.empty((B, ld), dtype=torch.float32, device="cuda")
+    idx = torch.empty((B, case.K), dtype=torch.int32, device="cuda")
+    out2 = torch.empty_like(lay.out)
+    tk_ws_n = _lib.topk_workspace_bytes(B, case.K, lay.max_len)
+    tk_ws = torch.empty(max(tk_ws_n, 256), dtype=torch.uint8, device="cuda")
+    at_ws_n = _lib.sparse_attn_workspace_bytes(B, case.H, case.K, case.Dv)
+    at_ws = torch.empty(max(at_ws_n, 256), dtype=torch.uint8, device="cuda")
+    K_st = max(20, args.steps // 2)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K_st)]
+    for it in range(K_st + 3):
+        flush.zero_()
+        e = ev[it - 3] if it >= 3 else None
+        if e: e[0].record(stream)
+        _lib.indexer_scores(lay.q_idx, lay.w, lay.k_cache, lay.pg, None, None, lay.max_len, scores)
+        if e: e[1].record(stream)
+        _lib.topk(scores, lay.seq_lens, case.K, lay.max_len, idx=idx, ws=tk_ws)
+        if e: e[2].record(stream)
+        _lib.sparse_attn(lay.q, lay.kv_cache, lay.pg, None, idx, lay.gate, case.sm_scale, case.Dv, out=out2, ws=at_ws)
+        if e: e[3].record(stream)
+    torch.cuda.synchronize()
+    st = {k: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev) * 1e3
+          for i, k in enumerate(["indexer", "topk", "attention"])}
+
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    layer_bytes, idx_bytes = decode_bytes(case)
+    idx_gbs = idx_bytes / (st["indexer"] * 1e-6) / 1e9
+    traffic, traffic_src = profiled_traffic()
+    roofline = {"bound": "hbm", "kernel": "indexer_decode_kernel<128,32> (dsa_indexer_scores)",
+                "achieved": round(idx_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(idx_gbs / hbm, 4),
+                "traffic": traffic, "traffic_source": traffic_src,
+                "algorithmic_bytes_per_launch": idx_bytes, "launch_us": round(st["indexer"], 2),
+                "peak_source": f"hbm_gbs, {peak_src}"}
+    step_mean_ms = total_ms / args.steps
+    layer_gbs = layer_bytes / (step_mean_ms * 1e-3) / 1e9
+
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 indexer / bf16 attention, fp32 accumulate",
+        "data": "synthetic (seeded; dyadic FP8 indexer operands, N(0,1) bf16 latent/q/gate)",
+        "config": {"workload": case.name, "batch_per_gpu": B, "context": Lctx, "indexer_heads": case.HI,
+                   "indexer_dim": case.DI, "top_k": case.K, "q_heads": case.H, "latent_dim": case.Dqk,
+                   "value_dim": case.Dv, "page_size": case.page_size,
+                   "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
+                   "l2": "flushed between timed steps (256 MiB write, outside the step events)"},
+        "roofline": roofline,
+        "layer_roofline": {"bound": "hbm", "algorithmic_bytes_per_step": layer_bytes,
+                           "achieved": round(layer_gbs, 1), "peak": hbm, "unit": "GB/s",
+                           "frac": round(layer_gbs / hbm, 4)},
+        "stages_us": {k: round(v, 2) for k, v in st.items()},
+        "gpu_launches": launches * args.steps,
+        "gpu_launches_per_step": launches,
+        "clocks": clk.summary(),
+    }
+
+    if not args.no_extras:
+        res["e2e"] = e2e_leg(args, lay, flush, stream, _lib)
+        if world == 1 and rank == 0:
+            res["prefill_indexer"] = prefill_indexer_leg(args, flush)
+            res["cpu_baseline"], orc_idx, orc_out = cpu_baseline_leg(case)
+            got_idx = lay.idx.cpu().numpy()
+            got = lay.out.float().cpu().numpy().astype(np.float64)
+            res["parity"] = {"idx_bit_exact": bool(np.array_equal(got_idx, orc_idx)),
+                             "out_max_abs_err": float(np.abs(got - orc_out).max()),
+                             "out_rel_fro_err": float(np.linalg.norm(got - orc_out) / np.linalg.norm(orc_out))}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+def e2e_leg(args, lay, flush, stream, _lib):
+    """The same decode step through dsa_layer_forward with the step's inputs
+    coming from pinned host memory and its output going back to it."""
+    import torch
+    K = max(20, args.steps // 2)
+    ins = [lay.q_idx, lay.w, lay.q, lay.gate, lay.seq_lens]
+    host_in = [t.cpu().pin_memory() for t in ins]
+    host_out = torch.empty(lay.out.shape, dtype=lay.out.dtype).pin_memory()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K + 3)]
+    for i, (s, e) in enumerate(ev):
+        flush.zero_()
+        s.record(stream)
+        for d, h in zip(ins, host_in):
+            d.copy_(h, non_blocking=True)
+        lay.forward()
+        host_out.copy_(lay.out, non_blocking=True)
+        e.record(stream)
+    torch.cuda.synchronize()
+    ms = sum(s.elapsed_time(e) for s, e in ev[3:])
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+    return {"value": round(lay.case.T * K / (ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms / K, 5),
+            "note": "dsa_layer_forward; per-step inputs (q, qI, w, gate, seq_lens) pinned-host->device, "
+                    "out device->pinned-host inside the events; caches stay resident"}
+
+
+def fp8_peak_tflops():
+    """Dense e4m3 GEMM peak measured with torch._scaled_mm (8192^3, best of 10):
+    a library measuring stick for the prefill indexer's roofline."""
+    import torch
+    n = 8192
+    a = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn).t()
+    one = torch.ones((), device="cuda")
+    for _ in range(3):
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    best = float("inf")
+    for _ in range(10):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        e.record()
+        torch.cuda.synchronize()
+        best = min(best, s.elapsed_time(e))
+    return 2 * n ** 3 / (best * 1e-3) / 1e12
+
+
+def prefill_indexer_leg(args, flush, T=32768):
+    import numpy as np
+    import torch
+    from long_context_sparse_02_b200 import _lib, synth
+    from long_context_sparse_02_b200.runtime import to_dev
+    rng = np.random.default_rng(args.seed + 7)
+    HI, DI = 16, 128
+    ss = np.random.SeedSequence(args.seed + 7).spawn(3)
+    bt, npg = synth.paged_layout(np.random.default_rng(ss[0]), [T])
+    q_idx = to_dev(synth.dyadic_e4m3(np.random.default_rng(ss[1]), (T, HI, DI)))
+    k_cache = to_dev(synth.dyadic_e4m3(np.random.default_rng(ss[2]), (npg, 64, DI)))
+    w = to_dev(synth.dyadic_weights(rng, (T, HI)))
+    seq_lens = to_dev(np.array([T], np.int32))
+    pg = _lib.paged(seq_lens, to_dev(bt), npg)
+    q_seq = torch.zeros(T, dtype=torch.int32, device="cuda")
+    q_pos = torch.arange(T, dtype=torch.int32, device="cuda")
+    scores = torch.empty((T, T), dtype=torch.float32, device="cuda")
+    call = lambda: _lib.indexer_scores(q_idx, w, k_cache, pg, q_seq, q_pos, T, scores)  # noqa: E731
+    for _ in range(3):
+        call()
+    ms = []
+    for _ in range(10):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        call()
+        e.record()
+        torch.cuda.synchronize()
+        ms.append(s.elapsed_time(e))
+    t = statistics.median(ms)
+    flops = 2.0 * HI * DI * T * (T + 1) / 2
+    peak = fp8_peak_tflops()
+    tf = flops / (t * 1e-3) / 1e12
+    del scores
+    torch.cuda.empty_cache()
+    return {"workload": f"prefill_T{T}_indexer_{HI}x{DI}", "ms": round(t, 4), "tflops": round(tf, 1),
+            "fp8_peak_tflops": round(peak, 1), "frac": round(tf / peak, 4), "bound": "tensor",
+            "peak_source": "measured in this run: torch._scaled_mm e4m3 8192^3, best of 10",
+            "algorithmic_flops": flops}
+
+
+def cpu_baseline_leg(case):
+    """The oracle as it stands on this host: one whole decode step of the
+    workload (every sequence, full context, all heads)."""
+    import numpy as np
+    from oracle import oracle
+    pg = oracle.Paged(case.seq_lens, case.block_table, case.page_size, case.num_pages)
+    t0 = time.perf_counter()
+    _, idx, out = oracle.layer_forward(case.q_idx, case.w, case.k_cache, case.q, case.kv_cache, case.gate, pg,
+                                       np.arange(case.T, dtype=np.int32), case.seq_lens - 1, case.K, case.Dv,
+                                       case.sm_scale)
+    dt = time.perf_counter() - t0
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    cores = int(os.environ.get("OMP_NUM_THREADS", cores))
+    return ({"value": round(case.T / dt, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+             "seconds": round(dt, 2),
+             "sample": f"one full decode step of {case.name} ({case.T} sequences x {case.max_len} tokens, "
+                       f"all heads) through oracle.c (fp64, OpenMP)"}, idx, out)
+
+
+# ---------------------------------------------------------------- reference arm (the oracle)
+
+def run_reference(args):
+    """--impl reference: the CPU oracle, as it stands, on this host's cores.
+    Each step is a bounded sample of one decode token: 1/F of its keys and
+    1/F of its heads (F a power of two sized so the run fits the budget);
+    throughput is scaled back by F."""
+    import numpy as np
+    from long_context_sparse_02_b200 import synth
+    from oracle import oracle
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    oracle.build()
+    B, Lctx = args.batch, args.context
+
+    def sample(F, seed):
+        L = max(Lctx // F, 64)
+        H = max(128 // F, 1)
+        return synth.decode_case(seed, [L], HI=32, H=H, name=f"decode_1of{F}")
+
+    def step(c):
+        pg = oracle.Paged(c.seq_lens, c.block_table, c.page_size, c.num_pages)
+        t0 = time.perf_counter()
+        oracle.layer_forward(c.q_idx, c.w, c.k_cache, c.q, c.kv_cache, c.gate, pg, np.zeros(1, np.int32),
+                             c.seq_lens - 1, c.K, c.Dv, c.sm_scale)
+        return time.perf_counter() - t0
+
+    probe = sample(16, args.seed)
+    t16 = step(probe)
+    per_step = args.ref_budget_s / max(1, args.steps + args.warmup)
+    F = 1
+    while F < 128 and t16 * 16 / F > per_step:
+        F *= 2
+    c = sample(F, args.seed)
+    for _ in range(args.warmup):
+        step(c)
+    times = [step(c) for _ in range(args.steps)]
+    total = sum(times)
+    value = (args.steps / F) / total
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    sample_desc = (f"per step: one decode token with 1/{F} of its work -- {c.max_len} of {Lctx} keys through "
+                   f"the 32x128 indexer and top-2048, {c.H} of 128 heads of attention; tokens/s scaled by 1/{F}")
+    res = {"metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+           "config": {"workload": f"decode_B{B}_L{Lctx}", "batch_per_gpu": B, "context": Lctx},
+           "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": cores, "kind": "oracle",
+                            "sample": sample_desc},
+           "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse_args()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_native(a)

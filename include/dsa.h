@@ -163,6 +163,10 @@ size_t dsa_layer_workspace_bytes(const dsa_layer_args *a);
 dsa_status dsa_layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes,
                              dsa_stream_t stream);
 
+/* Number of kernels dsa_layer_forward launches for these arguments (host
+ * only; the top-K scratch reset is a memset and is not counted). */
+int32_t dsa_layer_kernel_launches(const dsa_layer_args *a);
+
 /* ---- sliding-window decode (the hybrid's local layers) ------------------------
  * "aiany.app item naive-n0-5-flash", Key Capabilities: 5 sliding-window
  * layers (window 128) per DSA layer.  Sequence b's query (position

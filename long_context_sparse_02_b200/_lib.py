@@ -73,12 +73,14 @@ lib.dsa_layer_workspace_bytes.restype = SZ
 lib.dsa_layer_workspace_bytes.argtypes = [ctypes.POINTER(LayerArgs)]
 lib.dsa_layer_forward.restype = ctypes.c_int
 lib.dsa_layer_forward.argtypes = [ctypes.POINTER(LayerArgs), P, SZ, P]
+lib.dsa_layer_kernel_launches.restype = I32
+lib.dsa_layer_kernel_launches.argtypes = [ctypes.POINTER(LayerArgs)]
 lib.dsa_swa_decode.restype = ctypes.c_int
 lib.dsa_swa_decode.argtypes = [P, P, P, P, I32, I32, I32, I32, F32, P, P]
 
 EXPORTS = ["dsa_abi_version", "dsa_status_string", "dsa_device_error", "dsa_indexer_scores",
            "dsa_topk_workspace_bytes", "dsa_topk", "dsa_sparse_attn_workspace_bytes", "dsa_sparse_attn",
-           "dsa_layer_workspace_bytes", "dsa_layer_forward", "dsa_swa_decode"]
+           "dsa_layer_workspace_bytes", "dsa_layer_forward", "dsa_layer_kernel_launches", "dsa_swa_decode"]
 
 
 def _check(fn: str, status: int):
@@ -187,6 +189,10 @@ def layer_args(mode, q_idx, w, k_cache, q, kv_cache, gate, pg: Paged, q_seq, q_p
 
 def layer_workspace_bytes(args: LayerArgs) -> int:
     return int(lib.dsa_layer_workspace_bytes(ctypes.byref(args)))
+
+
+def layer_kernel_launches(args: LayerArgs) -> int:
+    return int(lib.dsa_layer_kernel_launches(ctypes.byref(args)))
 
 
 def layer_forward(args: LayerArgs, ws: torch.Tensor):

@@ -251,6 +251,11 @@ dsa_status dsa_layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes,
     return launch_attn(aa, st);
 }
 
+int32_t dsa_layer_kernel_launches(const dsa_layer_args *a) {
+    if (!a || a->T <= 0 || a->max_len < 1) return 0;
+    return 1 + topk_kernel_launches(a->max_len) + attn_kernel_launches(a->T, a->K, a->Dv);
+}
+
 dsa_status dsa_swa_decode(const uint16_t *q, const uint16_t *k_ring, const uint16_t *v_ring, const int32_t *seq_lens,
                           int32_t B, int32_t H, int32_t D, int32_t window, float sm_scale, uint16_t *out,
                           dsa_stream_t stream) {

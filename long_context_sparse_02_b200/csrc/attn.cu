@@ -502,6 +502,12 @@ size_t attn_workspace_bytes(int32_t T, int32_t H, int32_t K, int32_t Dv) {
     return align_up(rows * Dv * 4, 256) + align_up(rows * 2 * 4, 256);
 }
 
+int attn_kernel_launches(int32_t T, int32_t K, int32_t Dv) {
+    const DeviceInfo *dev = current_device();
+    if (!dev || T <= 0) return 0;
+    return plan_for(T, K, Dv, dev->sm_count).splits > 1 ? 2 : 1;
+}
+
 dsa_status launch_attn(const AttnArgs &a, cudaStream_t st) {
     const DeviceInfo *dev = current_device();
     if (!dev) return DSA_ERR_CUDA;

@@ -61,6 +61,7 @@ struct TopkArgs {
     size_t ws_bytes;
 };
 size_t topk_workspace_bytes(int32_t R, int32_t K, int32_t max_row_len);
+int topk_kernel_launches(int32_t max_row_len);
 dsa_status launch_topk(const TopkArgs &a, cudaStream_t st);
 
 // ---- gated sparse attention ----------------------------------------------------
@@ -80,6 +81,7 @@ struct AttnArgs {
     size_t ws_bytes;
 };
 size_t attn_workspace_bytes(int32_t T, int32_t H, int32_t K, int32_t Dv);
+int attn_kernel_launches(int32_t T, int32_t K, int32_t Dv);
 dsa_status launch_attn(const AttnArgs &a, cudaStream_t st);
 
 // ---- sliding-window decode -------------------------------------------------------

@@ -337,6 +337,8 @@ size_t topk_workspace_bytes(int32_t R, int32_t K, int32_t max_row_len) {
     return align_up(multi_zero_bytes(R) + (size_t)R * nch * 2 * 4, 256);
 }
 
+int topk_kernel_launches(int32_t max_row_len) { return max_row_len <= SMALL_CAP ? 1 : 5; }
+
 dsa_status launch_topk(const TopkArgs &a, cudaStream_t st) {
     const DeviceInfo *dev = current_device();
     if (!dev) return DSA_ERR_CUDA;
