@@ -109,6 +109,34 @@ dsa_status dsa_topk(const float *scores, int64_t ld, const int32_t *row_len,
                     int32_t R, int32_t K, int32_t max_row_len, int32_t *idx,
                     void *ws, size_t ws_bytes, dsa_stream_t stream);
 
+/* ---- top-K with library-owned scratch ---------------------------------------
+ * Not described by the source pages: an interface addition for callers that
+ * cannot allocate device memory where the selection runs -- an engine whose
+ * GPU memory is reserved up front by its own pool (a cudaMalloc would fail or
+ * fragment that pool), or a latency-bound decode loop that cannot afford
+ * cudaMalloc's implicit device-wide synchronisation.
+ * Same result as dsa_topk (same arguments minus the workspace), computed by
+ * the multi-CTA selection kernels on a scratch array the library holds in
+ * each GPU's memory for the life of the process (DSA_TOPK_STATIC_SCRATCH_BYTES,
+ * about 417 KB).  It allocates and frees nothing.
+ *  - Limits: R <= DSA_TOPK_STATIC_MAX_ROWS and max_row_len <=
+ *    DSA_TOPK_STATIC_MAX_ROW_LEN; larger calls return DSA_ERR_UNSUPPORTED
+ *    before launching anything.
+ *  - The first call on a device looks up the scratch array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture begins.
+ *  - Every call on a device shares the one array, which keeps the previous
+ *    call's contents; each call clears what must start at zero.  Calls whose
+ *    GPU work overlaps (different streams, no ordering between them) race on
+ *    the array and give wrong results: order them on one stream or with
+ *    events. */
+#define DSA_TOPK_STATIC_MAX_ROWS 16
+#define DSA_TOPK_STATIC_MAX_ROW_LEN 1048576
+#define DSA_TOPK_STATIC_SCRATCH_BYTES 426496
+dsa_status dsa_topk_static(const float *scores, int64_t ld, const int32_t *row_len,
+                           int32_t R, int32_t K, int32_t max_row_len, int32_t *idx,
+                           dsa_stream_t stream);
+
 /* ---- stage 3: gated attention over the selected latent rows ----------------
  * For query t, head h, and the selected rows c_j = latent row idx[t*K + j] of
  * sequence q_seq[t] (entries < 0 are padding):

@@ -64,6 +64,8 @@ lib.dsa_topk_workspace_bytes.restype = SZ
 lib.dsa_topk_workspace_bytes.argtypes = [I32, I32, I32]
 lib.dsa_topk.restype = ctypes.c_int
 lib.dsa_topk.argtypes = [P, I64, P, I32, I32, I32, P, P, SZ, P]
+lib.dsa_topk_static.restype = ctypes.c_int
+lib.dsa_topk_static.argtypes = [P, I64, P, I32, I32, I32, P, P]
 lib.dsa_sparse_attn_workspace_bytes.restype = SZ
 lib.dsa_sparse_attn_workspace_bytes.argtypes = [I32, I32, I32, I32]
 lib.dsa_sparse_attn.restype = ctypes.c_int
@@ -79,7 +81,8 @@ lib.dsa_swa_decode.restype = ctypes.c_int
 lib.dsa_swa_decode.argtypes = [P, P, P, P, I32, I32, I32, I32, F32, P, P]
 
 EXPORTS = ["dsa_abi_version", "dsa_status_string", "dsa_device_error", "dsa_indexer_scores",
-           "dsa_topk_workspace_bytes", "dsa_topk", "dsa_sparse_attn_workspace_bytes", "dsa_sparse_attn",
+           "dsa_topk_workspace_bytes", "dsa_topk", "dsa_topk_static", "dsa_sparse_attn_workspace_bytes",
+           "dsa_sparse_attn",
            "dsa_layer_workspace_bytes", "dsa_layer_forward", "dsa_layer_kernel_launches", "dsa_swa_decode"]
 
 

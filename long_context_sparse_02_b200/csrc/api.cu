@@ -192,6 +192,17 @@ dsa_status dsa_topk(const float *scores, int64_t ld, const int32_t *row_len, int
     return launch_topk(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+dsa_status dsa_topk_static(const float *scores, int64_t ld, const int32_t *row_len, int32_t R, int32_t K,
+                           int32_t max_row_len, int32_t *idx, dsa_stream_t stream) {
+    if (R < 0 || K < 1 || max_row_len < 1 || ld < max_row_len) return DSA_ERR_INVALID_ARG;
+    if (K > 4096 || R > DSA_TOPK_STATIC_MAX_ROWS || max_row_len > DSA_TOPK_STATIC_MAX_ROW_LEN)
+        return DSA_ERR_UNSUPPORTED;
+    if (R == 0) return DSA_OK;
+    if (!scores || !row_len || !idx) return DSA_ERR_INVALID_ARG;
+    TopkArgs a{scores, ld, row_len, ROWLEN_ARRAY, R, K, max_row_len, idx, nullptr, 0};
+    return launch_topk_static(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t dsa_sparse_attn_workspace_bytes(int32_t T, int32_t H, int32_t K, int32_t Dv) {
     if (T <= 0 || H <= 0 || K < 64) return 0;
     return attn_workspace_bytes(T, H, K, Dv);

@@ -16,6 +16,8 @@
 //   * longer rows: CHUNK-key slices per CTA, per-row global histograms, the
 //     last CTA of a pass (atomic ticket, no waiting) picks the digit; then a
 //     count pass and an offset-and-write pass.
+#include <mutex>
+
 #include "dsa_device.cuh"
 #include "dsa_internal.h"
 
@@ -353,6 +355,59 @@ dsa_status launch_topk(const TopkArgs &a, cudaStream_t st) {
     if (a.ws == nullptr || a.ws_bytes < need) return DSA_ERR_WORKSPACE;
     MultiWs m = carve_multi(a.ws, a.R, a.max_row_len);
     if (cudaMemsetAsync(a.ws, 0, multi_zero_bytes(a.R), st) != cudaSuccess) return DSA_ERR_CUDA;
+    dim3 grid(m.nchunks, a.R);
+    for (int ps = 0; ps < 3; ++ps) topk_pass_kernel<<<grid, MULTI_THREADS, 0, st>>>(a, m, ps, dev->err);
+    topk_count_kernel<<<grid, MULTI_THREADS, 0, st>>>(a, m);
+    topk_write_kernel<<<grid, MULTI_THREADS, 0, st>>>(a, m, dev->err);
+    return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Top-K without caller-provided scratch.
+//
+// Some callers cannot allocate device memory on the path that selects
+// positions: an engine whose GPU memory is reserved up front by its own pool
+// (so a cudaMalloc would fail or fragment that pool), or a latency-bound
+// decode loop that cannot afford cudaMalloc's implicit device-wide
+// synchronisation.  For them the multi-CTA selection above runs on a scratch
+// area that lives in this library's own device memory: a file-scope array
+// every GPU that loads the library holds until the process exits.  Host code
+// cannot use the array's name as a device address, so its address is looked
+// up once per device with cudaGetSymbolAddress (with that device current) on
+// the first call.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int STATIC_MAX_ROWS = DSA_TOPK_STATIC_MAX_ROWS;
+constexpr int STATIC_MAX_ROW_LEN = DSA_TOPK_STATIC_MAX_ROW_LEN;
+constexpr size_t STATIC_SCRATCH_BYTES =
+    (size_t)STATIC_MAX_ROWS * (3 * HBINS * 4 + sizeof(RowState)) +
+    (size_t)STATIC_MAX_ROWS * ((STATIC_MAX_ROW_LEN + CHUNK - 1) / CHUNK) * 2 * 4;
+static_assert(STATIC_SCRATCH_BYTES == DSA_TOPK_STATIC_SCRATCH_BYTES, "header states the scratch size");
+
+static __device__ __align__(256) uint8_t g_topk_static_scratch[STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDev = 64;
+std::once_flag g_static_once[kMaxDev];
+void *g_static_ptr[kMaxDev];
+cudaError_t g_static_rc[kMaxDev];
+}  // namespace
+
+dsa_status launch_topk_static(const TopkArgs &a, cudaStream_t st) {
+    const DeviceInfo *dev = current_device();
+    if (!dev || dev->device >= kMaxDev) return DSA_ERR_CUDA;
+    if (a.R > STATIC_MAX_ROWS || a.max_row_len > STATIC_MAX_ROW_LEN) return DSA_ERR_UNSUPPORTED;
+    if (a.R == 0) return DSA_OK;
+    const int d = dev->device;
+    std::call_once(g_static_once[d], [d] {
+        void *p = nullptr;
+        g_static_rc[d] = cudaGetSymbolAddress(&p, g_topk_static_scratch);
+        g_static_ptr[d] = p;
+    });
+    if (g_static_rc[d] != cudaSuccess || !g_static_ptr[d]) return DSA_ERR_CUDA;
+    MultiWs m = carve_multi(g_static_ptr[d], a.R, a.max_row_len);
+    // Histograms, tickets and row state must start at zero; the array keeps
+    // whatever the previous call left.
+    if (cudaMemsetAsync(g_static_ptr[d], 0, multi_zero_bytes(a.R), st) != cudaSuccess) return DSA_ERR_CUDA;
     dim3 grid(m.nchunks, a.R);
     for (int ps = 0; ps < 3; ++ps) topk_pass_kernel<<<grid, MULTI_THREADS, 0, st>>>(a, m, ps, dev->err);
     topk_count_kernel<<<grid, MULTI_THREADS, 0, st>>>(a, m);
