@@ -39,6 +39,21 @@ METRIC = "DSA-layer decode tokens/s @128K ctx; prefill indexer TFLOPS & % HBM/FP
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20   # > 126 MB L2
+
+
+class L2Flush:
+    """Evicts the step's data from L2 between timed steps: writes a buffer
+    larger than L2, then reads another one, so the dirty lines of the write
+    are written back here and not inside the next timed step."""
+
+    def __init__(self):
+        import torch
+        self.w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        self.r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    def zero_(self):
+        self.w.zero_()
+        self.r.sum()
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "indexer_decode_B8_L131072.md")
 
 
@@ -57,6 +72,8 @@ def parse_args(argv=None):
                     help="skip the prefill-indexer, e2e, CPU-baseline and parity legs (profiling runs)")
     ap.add_argument("--ref-budget-s", type=float, default=120.0,
                     help="wall-clock budget of the --impl reference run")
+    ap.add_argument("--prefill-only", type=int, default=0, metavar="T",
+                    help="time only the prefill indexer at T queries (small cases for profiling)")
     return ap.parse_args(argv)
 
 
@@ -216,7 +233,7 @@ def run_native(args):
     case = synth.decode_case(args.seed + 1000 * rank, [Lctx] * B, HI=32, name=f"decode_B{B}_L{Lctx}")
     lay = LayerOnDevice(case, decode=True, want_idx=True)
     launches = _lib.layer_kernel_launches(lay.args)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
     stream = torch.cuda.current_stream()
     _lib.device_error(reset=True)
 
@@ -230,54 +247,41 @@ def run_native(args):
         lay.forward()
     barrier()
 
-    # ---- timed region: K steps of dsa_layer_forward, L2 flushed between steps
-    def timed(fn, K):
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    # ---- timed region: K steps of the layer through the C ABI, L2 flushed
+    # between steps.  dsa_layer_forward_profiled is dsa_layer_forward plus four
+    # event records (before the indexer, after it, after top-K, after the
+    # attention), so the stage split comes from the timed steps themselves.
+    def make_events(K):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+        for e4 in ev:
+            for e in e4:
+                e.record(stream)  # creates the handle
+        torch.cuda.synchronize()
+        return ev
+
+    def timed(K):
+        ev = make_events(K)
         barrier()
-        for s, e in ev:
+        for e4 in ev:
             flush.zero_()
-            s.record(stream)
-            fn()
-            e.record(stream)
+            lay.forward_profiled(e4)
         barrier()
-        return [s.elapsed_time(e) for s, e in ev]
+        return ev
 
     for attempt in range(2):
         clk = ClockSampler(local)
         with clk:
-            step_ms = timed(lay.forward, args.steps)
+            ev = timed(args.steps)
         if not clk.rejected():
             break
+    step_ms = [e4[0].elapsed_time(e4[3]) for e4 in ev]
     total_ms = sum(step_ms)
     err = _lib.device_error(reset=True)
     if err:
         raise RuntimeError(f"device error word {err:#x} after the timed region")
     max_ms, tokens = aggregate(total_ms, B * args.steps, world)
     value = tokens / (max_ms / 1e3)
-
-    # ---- per-stage split (the same kernels, one entry point each)
-    ld = (lay.max_len + 3) // 4 * 4
-    scores = torch.empty((B, ld), dtype=torch.float32, device="cuda")
-    idx = torch.empty((B, case.K), dtype=torch.int32, device="cuda")
-    out2 = torch.empty_like(lay.out)
-    tk_ws_n = _lib.topk_workspace_bytes(B, case.K, lay.max_len)
-    tk_ws = torch.empty(max(tk_ws_n, 256), dtype=torch.uint8, device="cuda")
-    at_ws_n = _lib.sparse_attn_workspace_bytes(B, case.H, case.K, case.Dv)
-    at_ws = torch.empty(max(at_ws_n, 256), dtype=torch.uint8, device="cuda")
-    K_st = max(20, args.steps // 2)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K_st)]
-    for it in range(K_st + 3):
-        flush.zero_()
-        e = ev[it - 3] if it >= 3 else None
-        if e: e[0].record(stream)
-        _lib.indexer_scores(lay.q_idx, lay.w, lay.k_cache, lay.pg, None, None, lay.max_len, scores)
-        if e: e[1].record(stream)
-        _lib.topk(scores, lay.seq_lens, case.K, lay.max_len, idx=idx, ws=tk_ws)
-        if e: e[2].record(stream)
-        _lib.sparse_attn(lay.q, lay.kv_cache, lay.pg, None, idx, lay.gate, case.sm_scale, case.Dv, out=out2, ws=at_ws)
-        if e: e[3].record(stream)
-    torch.cuda.synchronize()
-    st = {k: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev) * 1e3
+    st = {k: statistics.mean(e4[i].elapsed_time(e4[i + 1]) for e4 in ev) * 1e3
           for i, k in enumerate(["indexer", "topk", "attention"])}
 
     peaks, peak_src = load_peaks()
@@ -285,7 +289,7 @@ def run_native(args):
     layer_bytes, idx_bytes = decode_bytes(case)
     idx_gbs = idx_bytes / (st["indexer"] * 1e-6) / 1e9
     traffic, traffic_src = profiled_traffic()
-    roofline = {"bound": "hbm", "kernel": "indexer_decode_kernel<128,32> (dsa_indexer_scores)",
+    roofline = {"bound": "hbm", "kernel": "indexer_decode_kernel<128,32> (stage 1 of dsa_layer_forward)",
                 "achieved": round(idx_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(idx_gbs / hbm, 4),
                 "traffic": traffic, "traffic_source": traffic_src,
                 "algorithmic_bytes_per_launch": idx_bytes, "launch_us": round(st["indexer"], 2),
@@ -302,7 +306,8 @@ def run_native(args):
                    "indexer_dim": case.DI, "top_k": case.K, "q_heads": case.H, "latent_dim": case.Dqk,
                    "value_dim": case.Dv, "page_size": case.page_size,
                    "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
-                   "l2": "flushed between timed steps (256 MiB write, outside the step events)"},
+                   "l2": "flushed between timed steps, outside the step events (256 MiB write, then a "
+                         "256 MiB read so no dirty lines remain)"},
         "roofline": roofline,
         "layer_roofline": {"bound": "hbm", "algorithmic_bytes_per_step": layer_bytes,
                            "achieved": round(layer_gbs, 1), "peak": hbm, "unit": "GB/s",
@@ -378,7 +383,7 @@ def fp8_peak_tflops():
     return 2 * n ** 3 / (best * 1e-3) / 1e12
 
 
-def prefill_indexer_leg(args, flush, T=32768):
+def prefill_indexer_leg(args, flush, T=32768, with_peak=True):
     import numpy as np
     import torch
     from long_context_sparse_02_b200 import _lib, synth
@@ -409,7 +414,7 @@ def prefill_indexer_leg(args, flush, T=32768):
         ms.append(s.elapsed_time(e))
     t = statistics.median(ms)
     flops = 2.0 * HI * DI * T * (T + 1) / 2
-    peak = fp8_peak_tflops()
+    peak = fp8_peak_tflops() if with_peak else float("nan")
     tf = flops / (t * 1e-3) / 1e12
     del scores
     torch.cuda.empty_cache()
@@ -495,5 +500,11 @@ if __name__ == "__main__":
     a = parse_args()
     if a.impl == "reference":
         run_reference(a)
+    elif a.prefill_only:
+        import torch
+        from long_context_sparse_02_b200 import build
+        build.build()
+        fl = L2Flush()
+        print(json.dumps(prefill_indexer_leg(a, fl, T=a.prefill_only, with_peak=False)))
     else:
         run_native(a)

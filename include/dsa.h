@@ -191,6 +191,13 @@ size_t dsa_layer_workspace_bytes(const dsa_layer_args *a);
 dsa_status dsa_layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes,
                              dsa_stream_t stream);
 
+/* dsa_layer_forward that also records caller-created CUDA events (cudaEvent_t
+ * handles; NULL entries are skipped) on `stream`: events[0] before the
+ * indexer, events[1] after it, events[2] after top-K, events[3] after the
+ * attention.  Same work, same launches; for timing the stages in place. */
+dsa_status dsa_layer_forward_profiled(const dsa_layer_args *a, void *ws, size_t ws_bytes,
+                                      void *const events[4], dsa_stream_t stream);
+
 /* Number of kernels dsa_layer_forward launches for these arguments (host
  * only; the top-K scratch reset is a memset and is not counted). */
 int32_t dsa_layer_kernel_launches(const dsa_layer_args *a);

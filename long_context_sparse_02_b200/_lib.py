@@ -75,6 +75,8 @@ lib.dsa_layer_workspace_bytes.restype = SZ
 lib.dsa_layer_workspace_bytes.argtypes = [ctypes.POINTER(LayerArgs)]
 lib.dsa_layer_forward.restype = ctypes.c_int
 lib.dsa_layer_forward.argtypes = [ctypes.POINTER(LayerArgs), P, SZ, P]
+lib.dsa_layer_forward_profiled.restype = ctypes.c_int
+lib.dsa_layer_forward_profiled.argtypes = [ctypes.POINTER(LayerArgs), P, SZ, ctypes.POINTER(P), P]
 lib.dsa_layer_kernel_launches.restype = I32
 lib.dsa_layer_kernel_launches.argtypes = [ctypes.POINTER(LayerArgs)]
 lib.dsa_swa_decode.restype = ctypes.c_int
@@ -83,7 +85,8 @@ lib.dsa_swa_decode.argtypes = [P, P, P, P, I32, I32, I32, I32, F32, P, P]
 EXPORTS = ["dsa_abi_version", "dsa_status_string", "dsa_device_error", "dsa_indexer_scores",
            "dsa_topk_workspace_bytes", "dsa_topk", "dsa_topk_static", "dsa_sparse_attn_workspace_bytes",
            "dsa_sparse_attn",
-           "dsa_layer_workspace_bytes", "dsa_layer_forward", "dsa_layer_kernel_launches", "dsa_swa_decode"]
+           "dsa_layer_workspace_bytes", "dsa_layer_forward", "dsa_layer_forward_profiled",
+           "dsa_layer_kernel_launches", "dsa_swa_decode"]
 
 
 def _check(fn: str, status: int):
@@ -201,6 +204,13 @@ def layer_kernel_launches(args: LayerArgs) -> int:
 def layer_forward(args: LayerArgs, ws: torch.Tensor):
     _check("dsa_layer_forward", lib.dsa_layer_forward(ctypes.byref(args), _ptr(ws, torch.uint8, "ws"),
                                                       ws.numel(), _stream()))
+
+
+def layer_forward_profiled(args: LayerArgs, ws: torch.Tensor, events):
+    """events: four recorded-once torch.cuda.Event objects (or None)."""
+    arr = (P * 4)(*[P(e.cuda_event) if e is not None else P(0) for e in events])
+    _check("dsa_layer_forward_profiled", lib.dsa_layer_forward_profiled(
+        ctypes.byref(args), _ptr(ws, torch.uint8, "ws"), ws.numel(), arr, _stream()))
 
 
 def swa_decode(q, k_ring, v_ring, seq_lens, window: int, sm_scale: float, out=None):

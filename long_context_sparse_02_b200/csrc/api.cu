@@ -227,7 +227,17 @@ size_t dsa_layer_workspace_bytes(const dsa_layer_args *a) {
     return carve_layer(a, nullptr).total;
 }
 
-dsa_status dsa_layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes, dsa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+dsa_status layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes, dsa_stream_t stream,
+                         void *const *events) {
+    auto mark = [&](int i) {
+        if (events && events[i])
+            return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), reinterpret_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess;
+        return true;
+    };
     if (!a) return DSA_ERR_INVALID_ARG;
     const bool decode = a->mode == DSA_MODE_DECODE;
     if (!decode && a->mode != DSA_MODE_PREFILL) return DSA_ERR_INVALID_ARG;
@@ -250,21 +260,38 @@ dsa_status dsa_layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes,
     const int64_t ld = (int64_t)ld_of(a->max_len);
     IndexerArgs ia{a->q_idx, a->w, a->k_idx_cache, pg, decode ? nullptr : a->q_seq, decode ? nullptr : a->q_pos,
                    a->T, a->HI, a->DI, a->max_len, lw.scores, ld};
+    if (!mark(0)) return DSA_ERR_CUDA;
     dsa_status s = launch_indexer(ia, st);
     if (s != DSA_OK) return s;
+    if (!mark(1)) return DSA_ERR_CUDA;
     TopkArgs ta{lw.scores, ld, decode ? a->pg.seq_lens : a->q_pos,
                 decode ? (int32_t)ROWLEN_SEQ_LENS : (int32_t)ROWLEN_QPOS_PLUS_1,
                 a->T, a->K, a->max_len, lw.idx, lw.topk_ws, lw.topk_bytes};
     s = launch_topk(ta, st);
     if (s != DSA_OK) return s;
+    if (!mark(2)) return DSA_ERR_CUDA;
     AttnArgs aa{a->q, a->kv_cache, pg, decode ? nullptr : a->q_seq, lw.idx, a->K, a->gate, a->sm_scale, a->T, a->H,
                 a->Dqk, a->Dv, a->out, a->lse, lw.attn_ws, lw.attn_bytes};
-    return launch_attn(aa, st);
+    s = launch_attn(aa, st);
+    if (s != DSA_OK) return s;
+    return mark(3) ? DSA_OK : DSA_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" {
+
+dsa_status dsa_layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes, dsa_stream_t stream) {
+    return layer_forward(a, ws, ws_bytes, stream, nullptr);
+}
+
+dsa_status dsa_layer_forward_profiled(const dsa_layer_args *a, void *ws, size_t ws_bytes, void *const events[4],
+                                      dsa_stream_t stream) {
+    return layer_forward(a, ws, ws_bytes, stream, events);
 }
 
 int32_t dsa_layer_kernel_launches(const dsa_layer_args *a) {
     if (!a || a->T <= 0 || a->max_len < 1) return 0;
-    return 1 + topk_kernel_launches(a->max_len) + attn_kernel_launches(a->T, a->K, a->Dv);
+    return 1 + topk_kernel_launches(a->T, a->max_len) + attn_kernel_launches(a->T, a->K, a->Dv);
 }
 
 dsa_status dsa_swa_decode(const uint16_t *q, const uint16_t *k_ring, const uint16_t *v_ring, const int32_t *seq_lens,

@@ -412,6 +412,380 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     }
 }
 
+// ============================================================================
+// Decode: one CTA = (query token, 128 selected rows).  The 128 gathered
+// latent rows stay resident in shared memory (all copies in flight at once);
+// Q streams from L2 through a small TMA ring.  S = Q C^T fills 128 TMEM
+// columns; the softmax over the 128 rows is exact (no running max); after S
+// has been read, O = P V overwrites TMEM columns [0, Dv) with V read MN-major
+// from the same resident rows.  Output: bf16 partial o/l plus (max, sum) per
+// (token, split, head), merged by attn_decode_combine_kernel.
+// ============================================================================
+constexpr int DEC_NR = 128;      // rows per CTA
+constexpr int DEC_WORKERS = 16;  // warps 0..15: gather, then softmax and epilogue
+constexpr int DEC_MMA_WARP = 16;
+constexpr int DEC_Q_WARP = 17;
+constexpr int DEC_THREADS = 18 * 32;
+constexpr int DEC_WORKER_THREADS = DEC_WORKERS * 32;
+
+template <int DQK, int DV>
+struct DecAttnCfg {
+    static constexpr int NKB = DQK / 64;           // 128-byte k-blocks per row
+    static constexpr int NVB = DV / 64;
+    static constexpr int KB_BYTES = DEC_NR * 128;  // one k-block of 128 rows
+    static constexpr int C_BYTES = NKB * KB_BYTES;
+    static constexpr int QS = NKB >= 4 ? 4 : NKB;  // Q ring stages
+    static constexpr int Q_STAGE = 128 * 128;      // [128 heads x 64 dims] bf16
+    static constexpr int Q_BYTES = QS * Q_STAGE;
+    static constexpr int P_BYTES = 2 * 128 * 128;  // [128 heads x 128 rows] bf16, two atoms
+    static constexpr int RING = Q_BYTES > P_BYTES ? Q_BYTES : P_BYTES;
+    static constexpr int TMEM_COLS = DV <= 128 ? 128 : DV <= 256 ? 256 : 512;
+    static constexpr int NBAR = NKB + 2 * QS + 4;
+    static constexpr int OUT_ROW = DV * 2 + 16;   // staged output row (padded: conflict-free)
+    static constexpr int OUT_BYTES = 128 * OUT_ROW;
+    static constexpr bool OUT_IN_C = OUT_BYTES <= C_BYTES;
+    static_assert(OUT_IN_C || OUT_BYTES <= RING, "output staging fits");
+    static constexpr int DPW = DV / 4;            // value dims per worker warp in the epilogue
+    static constexpr int SMEM = 1024 + C_BYTES + RING + 8 * NBAR + 8 * DEC_NR + 2 * 4 * 128 * 4 + 64;
+    static_assert(DV >= 64 && DV % 64 == 0 && DV <= 512, "value width");
+};
+
+struct DecAttnParams {
+    const uint16_t *kv;
+    PagedDev pg;
+    const int32_t *q_seq;
+    const int32_t *idx;
+    int32_t K;
+    float scale_log2;
+    int32_t T, H, Dv, splits;
+    uint16_t *part_o;  // [T, splits, H, Dv] bf16, normalised by the split's sum
+    float *part_ml;    // [T, splits, H, 2]  (max in log2 units, sum)
+    uint32_t *err;
+};
+
+// Warps 0..15 first gather the 128 rows (every copy in flight at once), then
+// share the softmax (warp w: heads 32(w%4).., rows 32(w/4)..) and the
+// epilogue (heads 32(w%4).., value dims DV/4 * (w/4)..).  Warp 16 issues the
+// MMAs and owns TMEM; warp 17 streams Q.
+template <int DQK, int DV>
+__global__ void __launch_bounds__(DEC_THREADS, 1)
+    attn_decode_kernel(const __grid_constant__ CUtensorMap qmap, const DecAttnParams p) {
+    using C = DecAttnCfg<DQK, DV>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    uint8_t *Cs = smem;              // [NKB][128 rows][128 B]
+    uint8_t *ring = Cs + C::C_BYTES;  // Q stages, later P
+    uint64_t *c_full = reinterpret_cast<uint64_t *>(ring + C::RING);  // [NKB]
+    uint64_t *q_full = c_full + C::NKB;                                 // [QS]
+    uint64_t *q_empty = q_full + C::QS;                                 // [QS]
+    uint64_t *s_full = q_empty + C::QS;
+    uint64_t *p_full = s_full + 1;
+    uint64_t *o_full = p_full + 1;
+    uint64_t *drain = o_full + 1;
+    int64_t *rowid = reinterpret_cast<int64_t *>(drain + 1);  // [128] cache row of each selected entry, -1 = none
+    float *red_m = reinterpret_cast<float *>(rowid + DEC_NR);  // [4][128] partial row maxima
+    float *red_l = red_m + 4 * 128;                            // [4][128] partial sums
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(red_l + 4 * 128);
+    int *any_valid = reinterpret_cast<int *>(tmem_slot + 1);
+    volatile int *abort_flag = any_valid + 1;
+
+    const int warp = warp_id(), lane = lane_id();
+    const int t = blockIdx.y, split = blockIdx.x;
+    const int row0 = split * DEC_NR;
+    const int row_end = min(p.K, row0 + DEC_NR);
+    int b = p.q_seq ? p.q_seq[t] : t;
+    const bool tok_ok = b >= 0 && b < p.pg.num_seqs;
+    const int L = tok_ok ? p.pg.seq_lens[b] : 0;
+    if (!tok_ok) b = 0;
+    AttnParams ap{};  // for latent_row()
+    ap.pg = p.pg;
+    ap.idx = p.idx;
+    ap.K = p.K;
+    ap.err = p.err;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::NKB; ++i) mbar_init(&c_full[i], DEC_WORKER_THREADS);
+        for (int i = 0; i < C::QS; ++i) {
+            mbar_init(&q_full[i], 1);
+            mbar_init(&q_empty[i], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(p_full, DEC_WORKERS);
+        mbar_init(o_full, 1);
+        mbar_init(drain, 1);
+        *any_valid = 0;
+        *abort_flag = 0;
+        if (!tok_ok) record_error(p.err, DSA_DEVERR_POSITION);
+        fence_mbar_init();
+        tma_prefetch_desc(&qmap);
+    }
+    if (warp == DEC_MMA_WARP) tmem_alloc(tmem_slot, C::TMEM_COLS);
+    __syncthreads();
+    // Q does not depend on the selection: start it while the rows are resolved.
+    if (warp == DEC_Q_WARP && lane == 0)
+        for (int kb = 0; kb < C::QS; ++kb) {
+            mbar_expect_tx(&q_full[kb], C::Q_STAGE);
+            tma_load_2d(ring + kb * C::Q_STAGE, &qmap, &q_full[kb], kb * 64, t * p.H);
+        }
+    if (threadIdx.x < DEC_NR) {  // resolve every selected row once, through the block table
+        const int64_t rid = tok_ok ? latent_row(ap, b, L, t, row0 + threadIdx.x, row_end, true) : -1;
+        rowid[threadIdx.x] = rid;
+        if (rid >= 0) *any_valid = 1;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const bool work = *any_valid != 0;
+
+    if (warp < DEC_WORKERS) {
+        const int wt = threadIdx.x;  // 0..511
+        // ---------------- gather: all 128 rows, every k-block, in flight at once ----------------
+        // Eight consecutive lanes copy one row's 128-byte k-block segment (a
+        // full line per 8 lanes); a thread serves rows rg and rg + 64.
+        {
+            const int c8 = wt & 7, rg = wt >> 3;
+            if (work) {
+                const int64_t src0 = rowid[rg], src1 = rowid[rg + 64];
+#pragma unroll 1
+                for (int kb = 0; kb < C::NKB; ++kb) {
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const int r = rg + 64 * q;
+                        const int64_t src = q ? src1 : src0;
+                        uint8_t *d = Cs + kb * C::KB_BYTES + r * 128 + ((c8 ^ (r & 7)) << 4);
+                        if (src >= 0) cp_async_16(d, p.kv + src * DQK + kb * 64 + c8 * 8);
+                        else *reinterpret_cast<uint4 *>(d) = make_uint4(0, 0, 0, 0);
+                    }
+                    cp_async_commit();
+                }
+                // signal each k-block as its copies land (groups complete in order)
+#define DSA_DEC_SIGNAL(KB)                                                    \
+    if (KB < C::NKB) {                                                         \
+        cp_async_wait<(C::NKB - 1 - (KB)) < 0 ? 0 : (C::NKB - 1 - (KB))>();    \
+        fence_proxy_async_smem();                                              \
+        mbar_arrive(&c_full[KB]);                                              \
+    }
+                DSA_DEC_SIGNAL(0) DSA_DEC_SIGNAL(1) DSA_DEC_SIGNAL(2) DSA_DEC_SIGNAL(3) DSA_DEC_SIGNAL(4)
+                DSA_DEC_SIGNAL(5) DSA_DEC_SIGNAL(6) DSA_DEC_SIGNAL(7) DSA_DEC_SIGNAL(8)
+#undef DSA_DEC_SIGNAL
+            }
+        }
+        // ---------------- softmax: warp w = (head quarter w%4, row block w/4) ----------------
+        const int qr = warp & 3, cb = warp >> 2;
+        const int head = 32 * qr + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(32 * qr) << 16;
+        float m = -INFINITY;
+        bool have_o = false;
+        // Every worker passes the same named barriers whatever happens; a
+        // timed-out wait in any warp turns the whole softmax off for all.
+        const bool s_ok = work && mbar_wait(s_full, 0, p.err, abort_flag);
+        const bool go = !named_bar_or(1, DEC_WORKER_THREADS, !s_ok) && work;
+        uint32_t sr[32];
+        uint32_t vm = 0;
+        if (go) {
+            tc_fence_after();
+            vm = __ballot_sync(0xffffffffu, rowid[32 * cb + lane] >= 0);
+            tmem_ld32(tmem + 32 * cb + lane_off, sr);
+            tmem_wait_ld();
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if ((vm >> i) & 1u) mx = fmaxf(mx, __uint_as_float(sr[i]) * p.scale_log2);
+            red_m[cb * 128 + head] = mx;
+        }
+        named_bar_sync(1, DEC_WORKER_THREADS);
+        if (go) {
+            m = fmaxf(fmaxf(red_m[head], red_m[128 + head]), fmaxf(red_m[256 + head], red_m[384 + head]));
+            uint32_t pk[16];
+            float ls = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+                const float p0 = ((vm >> i) & 1u) ? exp2f(__uint_as_float(sr[i]) * p.scale_log2 - m) : 0.f;
+                const float p1 = ((vm >> (i + 1)) & 1u) ? exp2f(__uint_as_float(sr[i + 1]) * p.scale_log2 - m) : 0.f;
+                pk[i / 2] = pack_bf16(p0, p1);
+                const __nv_bfloat162 bv = *reinterpret_cast<__nv_bfloat162 *>(&pk[i / 2]);
+                ls += __bfloat162float(bv.x) + __bfloat162float(bv.y);
+            }
+            red_l[cb * 128 + head] = ls;
+            // P columns 32cb..32cb+31 -> atom cb/2, 16-byte chunks 4*(cb%2) .. 4*(cb%2)+3
+            uint8_t *atom = ring + (cb >> 1) * 16384 + head * 128;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int cc = 4 * (cb & 1) + q;
+                *reinterpret_cast<uint4 *>(atom + ((cc ^ (head & 7)) << 4)) =
+                    make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full);
+            have_o = mbar_wait(o_full, 0, p.err, abort_flag);
+            tc_fence_after();
+        }
+        // ---------------- epilogue: warp w = (head quarter w%4, value dims DV/4 * (w/4)..) ----------------
+        // every partial sum written; S, P and the rows are consumed; O is read by all or by none
+        have_o = !named_bar_or(1, DEC_WORKER_THREADS, go && !have_o) && go;
+        const float l = have_o ? red_l[head] + red_l[128 + head] + red_l[256 + head] + red_l[384 + head] : 0.f;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const int d0 = cb * C::DPW;
+        uint8_t *stg = (C::OUT_IN_C ? Cs : ring) + head * C::OUT_ROW + d0 * 2;
+#pragma unroll 1
+        for (int c0 = 0; c0 < C::DPW; c0 += 16) {
+            uint32_t o[16];
+            if (have_o) {
+                tmem_ld16(tmem + d0 + c0 + lane_off, o);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) o[i] = 0u;
+            }
+#pragma unroll
+            for (int i = 0; i < 16; i += 8) {
+                uint4 v;
+                v.x = pack_bf16(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
+                v.y = pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+                v.z = pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+                v.w = pack_bf16(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+                *reinterpret_cast<uint4 *>(stg + (c0 + i) * 2) = v;
+            }
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, DEC_WORKER_THREADS);  // the whole staged row is written
+        const bool live = head < p.H;
+        const int64_t prow = ((int64_t)t * p.splits + split) * p.H + head;
+        if (cb == 0 && live) {
+            bulk_store(p.part_o + prow * p.Dv, (C::OUT_IN_C ? Cs : ring) + head * C::OUT_ROW, DV * 2);
+            bulk_commit();
+            p.part_ml[prow * 2 + 0] = m;
+            p.part_ml[prow * 2 + 1] = l;
+            bulk_wait_read_all();
+        }
+    } else if (warp == DEC_Q_WARP) {
+        // ---------------- rest of the Q stream (TMA, from L2) ----------------
+        if (lane == 0) {
+            int issued = C::QS;
+            if (work)
+                for (int kb = C::QS; kb < C::NKB; ++kb) {
+                    const int s = kb % C::QS;
+                    if (!mbar_wait(&q_empty[s], ((kb / C::QS) & 1) ^ 1, p.err, abort_flag)) break;
+                    mbar_expect_tx(&q_full[s], C::Q_STAGE);
+                    tma_load_2d(ring + s * C::Q_STAGE, &qmap, &q_full[s], kb * 64, t * p.H);
+                    ++issued;
+                }
+            if (!work)  // never leave a copy in flight behind
+                for (int kb = 0; kb < C::QS; ++kb) mbar_wait(&q_full[kb], 0, p.err, nullptr);
+        }
+    } else {
+        // ---------------- MMA issuer (warp 16) ----------------
+        if (lane == 0 && work) {
+            constexpr uint32_t ID_S = idesc(1, 1, 0, 0, DEC_NR, 128);
+            bool ok = true;
+            const uint32_t c0 = smem_u32(Cs), r0 = smem_u32(ring);
+            for (int kb = 0; ok && kb < C::NKB; ++kb) {
+                const int s = kb % C::QS;
+                if (!mbar_wait(&c_full[kb], 0, p.err, abort_flag) ||
+                    !mbar_wait(&q_full[s], (kb / C::QS) & 1, p.err, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16(tmem, sdesc(r0 + s * C::Q_STAGE + 32 * k, 16, 1024, SWZ_128B),
+                             sdesc(c0 + kb * C::KB_BYTES + 32 * k, 16, 1024, SWZ_128B), ID_S, (kb | k) != 0);
+                mma_commit(&q_empty[s]);
+            }
+            if (ok) mma_commit(s_full);
+            if (ok && mbar_wait(p_full, 0, p.err, abort_flag)) {
+                tc_fence_after();
+                for (int nb = 0; nb < C::NVB; nb += 4) {
+                    const int nblk = (C::NVB - nb) < 4 ? (C::NVB - nb) : 4;
+                    const uint32_t id_pv = idesc(1, 1, 0, 1, 64 * nblk, 128);
+#pragma unroll
+                    for (int k = 0; k < DEC_NR / 16; ++k)
+                        mma_bf16(tmem + nb * 64, sdesc(r0 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, SWZ_128B),
+                                 sdesc(c0 + nb * C::KB_BYTES + k * 2048, C::KB_BYTES, 1024, SWZ_128B), id_pv, k != 0);
+                }
+                mma_commit(o_full);
+            }
+            mma_commit(drain);
+            mbar_wait(drain, 0, p.err, nullptr);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == DEC_MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// One warp per (token, head, 256-wide slice of the value dims):
+// out = sigmoid(g) * sum_s w_s o_s with w_s = l_s 2^(m_s - M) / sum l 2^(m - M).
+// The split partials are loaded eight at a time before they are summed.
+constexpr int CMB_SLICE = 256;
+__global__ void __launch_bounds__(256) attn_decode_combine_kernel(const DecAttnParams p, const uint16_t *gate,
+                                                                  uint16_t *out, float *lse) {
+    const int nsl = (p.Dv + CMB_SLICE - 1) / CMB_SLICE;
+    const int wid = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (wid >= p.T * p.H * nsl) return;
+    const int sl = wid % nsl;
+    const int h = (wid / nsl) % p.H;
+    const int t = wid / (nsl * p.H);
+    const int S = p.splits;
+    float ms = -INFINITY, ls = 0.f;
+    if (lane < S) {
+        const float *ml = p.part_ml + (((int64_t)t * S + lane) * p.H + h) * 2;
+        ms = ml[0];
+        ls = ml[1];
+    }
+    float M = ls > 0.f ? ms : -INFINITY;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float wl = ls > 0.f ? ls * exp2f(ms - M) : 0.f;
+    float wsum = wl;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+    const float g = __bfloat162float(__ushort_as_bfloat16(gate[(int64_t)t * p.H + h]));
+    const float scale = wsum > 0.f ? (1.f / (1.f + __expf(-g))) / wsum : 0.f;
+    const float coef = wl * scale;
+    const int d0 = sl * CMB_SLICE + lane * 8;
+    const bool live = d0 < p.Dv;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const uint16_t *base = p.part_o + ((int64_t)t * S * p.H + h) * p.Dv + d0;
+    const int64_t sstride = (int64_t)p.H * p.Dv;
+    for (int s0 = 0; s0 < S; s0 += 8) {
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            v[u] = (live && s0 + u < S) ? *reinterpret_cast<const uint4 *>(base + (s0 + u) * sstride)
+                                        : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float c = __shfl_sync(0xffffffffu, coef, (s0 + u) & 31);
+            const float cc = s0 + u < S ? c : 0.f;
+            const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                acc[2 * i] = fmaf(cc, __uint_as_float(w4[i] << 16), acc[2 * i]);
+                acc[2 * i + 1] = fmaf(cc, __uint_as_float(w4[i] & 0xFFFF0000u), acc[2 * i + 1]);
+            }
+        }
+    }
+    if (live) {
+        uint4 o;
+        o.x = pack_bf16(acc[0], acc[1]);
+        o.y = pack_bf16(acc[2], acc[3]);
+        o.z = pack_bf16(acc[4], acc[5]);
+        o.w = pack_bf16(acc[6], acc[7]);
+        *reinterpret_cast<uint4 *>(out + ((int64_t)t * p.H + h) * p.Dv + d0) = o;
+    }
+    if (sl == 0 && lane == 0 && lse)
+        lse[(int64_t)t * p.H + h] = wsum > 0.f ? (M + __log2f(wsum)) * 0.69314718055994531f : -INFINITY;
+}
+
 // Merges split partials: out = sigmoid(g) * sum_s w_s o_s with
 // w_s = l_s 2^(m_s - M) / sum_s' l_s' 2^(m_s' - M).
 __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
@@ -493,9 +867,20 @@ dsa_status run_attn(const CUtensorMap &qm, const AttnParams &p, cudaStream_t st)
 
 }  // namespace
 
+// Few queries (decode): one CTA per (token, 128 selected rows) plus a
+// combine.  Many queries (prefill): the row-looping kernel above.
+constexpr int DEC_MAX_T = 64;
+bool use_decode(int T) { return T <= DEC_MAX_T; }
+int dec_splits(int K) { return (K + DEC_NR - 1) / DEC_NR; }
+size_t dec_ws_bytes(int T, int H, int K, int Dv) {
+    const size_t rows = (size_t)T * dec_splits(K) * H;
+    return align_up(rows * Dv * 2, 256) + align_up(rows * 2 * 4, 256);
+}
+
 size_t attn_workspace_bytes(int32_t T, int32_t H, int32_t K, int32_t Dv) {
     const DeviceInfo *dev = current_device();
     if (!dev || T <= 0 || K < 64) return 0;
+    if (use_decode(T)) return dec_ws_bytes(T, H, K, Dv);
     Plan pl = plan_for(T, K, Dv, dev->sm_count);
     if (pl.splits == 1) return 0;
     const size_t rows = (size_t)T * pl.splits * H;
@@ -505,13 +890,52 @@ size_t attn_workspace_bytes(int32_t T, int32_t H, int32_t K, int32_t Dv) {
 int attn_kernel_launches(int32_t T, int32_t K, int32_t Dv) {
     const DeviceInfo *dev = current_device();
     if (!dev || T <= 0) return 0;
+    if (use_decode(T)) return 2;
     return plan_for(T, K, Dv, dev->sm_count).splits > 1 ? 2 : 1;
+}
+
+template <int DQK, int DV>
+dsa_status run_attn_decode(const CUtensorMap &qm, const DecAttnParams &p, const uint16_t *gate, uint16_t *out,
+                           float *lse, cudaStream_t st) {
+    using C = DecAttnCfg<DQK, DV>;
+    auto fn = attn_decode_kernel<DQK, DV>;
+    if (!ensure_smem(reinterpret_cast<const void *>(fn), C::SMEM)) return DSA_ERR_CUDA;
+    fn<<<dim3(p.splits, p.T), DEC_THREADS, C::SMEM, st>>>(qm, p);
+    if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+    const int warps = p.T * p.H * ((p.Dv + CMB_SLICE - 1) / CMB_SLICE);
+    attn_decode_combine_kernel<<<(warps + 7) / 8, 256, 0, st>>>(p, gate, out, lse);
+    return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 dsa_status launch_attn(const AttnArgs &a, cudaStream_t st) {
     const DeviceInfo *dev = current_device();
     if (!dev) return DSA_ERR_CUDA;
     if (a.T == 0) return DSA_OK;
+    CUtensorMap qm;
+    if (!make_tmap_2d(&qm, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Dqk, (uint64_t)a.T * a.H, (uint64_t)a.Dqk * 2,
+                      64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return DSA_ERR_INVALID_ARG;
+    if (use_decode(a.T)) {
+        DecAttnParams dp{};
+        dp.kv = a.kv;
+        dp.pg = a.pg;
+        dp.q_seq = a.q_seq;
+        dp.idx = a.idx;
+        dp.K = a.K;
+        dp.scale_log2 = a.sm_scale * 1.4426950408889634f;
+        dp.T = a.T;
+        dp.H = a.H;
+        dp.Dv = a.Dv;
+        dp.splits = dec_splits(a.K);
+        dp.err = dev->err;
+        const size_t rows = (size_t)a.T * dp.splits * a.H;
+        if (!a.ws || a.ws_bytes < dec_ws_bytes(a.T, a.H, a.K, a.Dv)) return DSA_ERR_WORKSPACE;
+        dp.part_o = static_cast<uint16_t *>(a.ws);
+        dp.part_ml = reinterpret_cast<float *>(static_cast<uint8_t *>(a.ws) + align_up(rows * a.Dv * 2, 256));
+        if (a.Dqk == 576 && a.Dv == 512) return run_attn_decode<576, 512>(qm, dp, a.gate, a.out, a.lse, st);
+        if (a.Dqk == 64 && a.Dv == 64) return run_attn_decode<64, 64>(qm, dp, a.gate, a.out, a.lse, st);
+        return DSA_ERR_UNSUPPORTED;
+    }
     Plan pl = plan_for(a.T, a.K, a.Dv, dev->sm_count);
     AttnParams p{};
     p.kv = a.kv;
@@ -537,10 +961,6 @@ dsa_status launch_attn(const AttnArgs &a, cudaStream_t st) {
         p.part_o = static_cast<float *>(a.ws);
         p.part_ml = reinterpret_cast<float *>(static_cast<uint8_t *>(a.ws) + align_up(rows * a.Dv * 4, 256));
     }
-    CUtensorMap qm;
-    if (!make_tmap_2d(&qm, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Dqk, (uint64_t)a.T * a.H, (uint64_t)a.Dqk * 2,
-                      64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
-        return DSA_ERR_INVALID_ARG;
     if (a.Dqk == 576 && a.Dv == 512) return run_attn<576, 256>(qm, p, st);
     if (a.Dqk == 64 && a.Dv == 64) return run_attn<64, 64>(qm, p, st);
     return DSA_ERR_UNSUPPORTED;

@@ -61,7 +61,7 @@ struct TopkArgs {
     size_t ws_bytes;
 };
 size_t topk_workspace_bytes(int32_t R, int32_t K, int32_t max_row_len);
-int topk_kernel_launches(int32_t max_row_len);
+int topk_kernel_launches(int32_t R, int32_t max_row_len);
 dsa_status launch_topk(const TopkArgs &a, cudaStream_t st);
 dsa_status launch_topk_static(const TopkArgs &a, cudaStream_t st);
 

@@ -19,7 +19,9 @@
 //     persistent CTA takes whole query groups (snake order, costliest first)
 //     and streams the key tiles of the group's causal range.
 // Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (and TMEM owner),
-// warps 2..5 = epilogue (one TMEM lane quarter each).
+// then two epilogue warpgroups that take alternate tiles (each warp reads
+// one TMEM lane quarter), so one tile's TMEM read latency overlaps another's
+// arithmetic.
 #include "dsa_device.cuh"
 #include "dsa_internal.h"
 
@@ -96,20 +98,24 @@ struct IdxParams {
 // decode: keys x heads, one query per tile
 // ============================================================================
 
+// Two CTAs share each SM (two TMA-issuing producers keep more of HBM busy
+// than one producer with a deeper ring), each with its own TMEM slice.
 template <int DI, int NH>
 struct DecCfg {
-    static constexpr int STAGES = DI == 128 ? 8 : 12;
-    static constexpr int ACC = 4;
-    static constexpr int A_BYTES = 128 * DI;
-    static constexpr int B_BYTES = NH * DI;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int CTAS_PER_SM = 2;
+    static constexpr int STAGES = DI == 128 ? 6 : 12;  // key tiles in flight per CTA
+    static constexpr int EPI_GROUPS = 2;  // epilogue warpgroups, alternate tiles
+    static constexpr int ACC = NH <= 32 ? 8 : 4;  // TMEM: ACC * NH <= 256 columns per CTA
+    static constexpr int THREADS = 64 + 128 * EPI_GROUPS;
+    static constexpr int A_BYTES = 128 * DI;      // one key tile (two pages)
+    static constexpr int B_BYTES = NH * DI;       // one query's heads
     static constexpr int TMEM_COLS = pow2_cols(ACC * NH);
     static constexpr uint32_t SWZ = DI == 128 ? SWZ_128B : SWZ_64B;
     static constexpr uint32_t SBO = 8 * DI;
     static constexpr int MAXT = 1024;
-    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * ACC + 1);
-    static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + 4 * (MAXT + 1) + 16;
-    static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * ACC + 4 + 1);
+    static constexpr int SMEM = 1024 + STAGES * A_BYTES + 2 * B_BYTES + BAR_BYTES + 4 * (MAXT + 1) + 16;
+    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "tile alignment");
 };
 
 // Index t with tstart[t] <= g < tstart[t+1] (tstart non-decreasing, g < tstart[T]).
@@ -123,18 +129,21 @@ __device__ __forceinline__ int locate(const int32_t *tstart, int T, int64_t g) {
 }
 
 template <int DI, int NH>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(DecCfg<DI, NH>::THREADS, DecCfg<DI, NH>::CTAS_PER_SM)
     indexer_decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                           const IdxParams p) {
     using C = DecCfg<DI, NH>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    uint8_t *stages = smem;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::STAGES * C::STAGE_BYTES);
+    uint8_t *stages = smem;                                  // [STAGES][A_BYTES]
+    uint8_t *qbuf = smem + C::STAGES * C::A_BYTES;            // [2][B_BYTES]
+    uint64_t *full = reinterpret_cast<uint64_t *>(qbuf + 2 * C::B_BYTES);
     uint64_t *empty = full + C::STAGES;
     uint64_t *tfull = empty + C::STAGES;
     uint64_t *tempty = tfull + C::ACC;
-    uint64_t *drain = tempty + C::ACC;
+    uint64_t *qfull = tempty + C::ACC;   // [2]
+    uint64_t *qempty = qfull + 2;        // [2]
+    uint64_t *drain = qempty + 2;
     int32_t *tstart = reinterpret_cast<int32_t *>(drain + 1);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tstart + C::MAXT + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -150,6 +159,10 @@ __global__ void __launch_bounds__(192, 1)
         for (int a = 0; a < C::ACC; ++a) {
             mbar_init(&tfull[a], 1);
             mbar_init(&tempty[a], 4);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&qfull[i], 1);
+            mbar_init(&qempty[i], 1);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -187,39 +200,90 @@ __global__ void __launch_bounds__(192, 1)
     const int64_t hi = total * (blockIdx.x + 1) / gridDim.x;
     const int n = static_cast<int>(hi - lo);
 
-    if (warp == 0 && lane == 0 && n > 0) {
+    if (warp == 0 && n > 0) {
         // ---------------- producer ----------------
-        int t = locate(tstart, T, lo);
-        int j = static_cast<int>(lo - tstart[t]);
-        QInfo qi = query_info(t, p.q_seq, p.q_pos, p.pg, p.max_len, p.err);
-        int issued = 0;
-        for (int i = 0; i < n; ++i) {
-            const int s = i % C::STAGES;
-            const uint32_t ph = (i / C::STAGES) & 1;
-            if (!mbar_wait(&empty[s], ph ^ 1, p.err, abort_flag)) break;
-            uint8_t *A = stages + s * C::STAGE_BYTES;
-            uint8_t *B = A + C::A_BYTES;
-            const int pg0 = page_of(p.pg, qi.b, 2 * j, p.err);
-            const int pg1 = (2 * j + 1) * 64 <= qi.last ? page_of(p.pg, qi.b, 2 * j + 1, p.err) : -1;
-            const uint32_t bytes = C::B_BYTES + (pg0 >= 0 ? 64 * DI : 0) + (pg1 >= 0 ? 64 * DI : 0);
-            mbar_expect_tx(&full[s], bytes);
-            if (pg0 >= 0) tma_load_2d(A, &kmap, &full[s], 0, pg0 * 64);
-            if (pg1 >= 0) tma_load_2d(A + 64 * DI, &kmap, &full[s], 0, pg1 * 64);
-            tma_load_2d(B, &qmap, &full[s], 0, t * p.HI);
-            ++issued;
-            if (++j == tstart[t + 1] - tstart[t]) {
-                j = 0;
-                do { ++t; } while (t < T && tstart[t + 1] == tstart[t]);
-                if (t < T) qi = query_info(t, p.q_seq, p.q_pos, p.pg, p.max_len, p.err);
+        // The warp looks up the next 32 tiles' (query, pages) in parallel, one
+        // tile per lane, a window ahead of the tiles lane 0 is issuing, so no
+        // block-table load sits on the issue path.
+        auto lookup = [&](int i, int &tq, int &p0, int &p1) {
+            tq = -1, p0 = -1, p1 = -1;
+            if (i < n) {
+                const int64_t g = lo + i;
+                tq = locate(tstart, T, g);
+                const int j = static_cast<int>(g - tstart[tq]);
+                const QInfo qi = query_info(tq, p.q_seq, p.q_pos, p.pg, p.max_len, p.err);
+                p0 = page_of(p.pg, qi.b, 2 * j, p.err);
+                p1 = (2 * j + 1) * 64 <= qi.last ? page_of(p.pg, qi.b, 2 * j + 1, p.err) : -1;
             }
+        };
+        int tq, p0, p1;
+        lookup(lane, tq, p0, p1);
+        int issued = 0, qo = -1, tprev = -1;
+        bool ok = true;
+        for (int base = 0; ok && base < n; base += 32) {
+            int tq_n, p0_n, p1_n;
+            lookup(base + 32 + lane, tq_n, p0_n, p1_n);
+            const int cnt = min(32, n - base);
+            for (int k = 0; k < cnt; ++k) {
+                const int t = __shfl_sync(0xffffffffu, tq, k);
+                const int pg0 = __shfl_sync(0xffffffffu, p0, k);
+                const int pg1 = __shfl_sync(0xffffffffu, p1, k);
+                if (lane == 0) {
+                    const int i = base + k;
+                    if (t != tprev) {  // a new query: its heads go to the next q buffer
+                        tprev = t;
+                        ++qo;
+                        const int qb = qo & 1;
+                        if (mbar_wait(&qempty[qb], ((qo >> 1) & 1) ^ 1, p.err, abort_flag)) {
+                            mbar_expect_tx(&qfull[qb], C::B_BYTES);
+                            tma_load_2d(qbuf + qb * C::B_BYTES, &qmap, &qfull[qb], 0, t * p.HI);
+                        } else {
+                            ok = false;
+                        }
+                    }
+                    const int s = i % C::STAGES;
+                    const uint32_t ph = (i / C::STAGES) & 1;
+                    if (ok && mbar_wait(&empty[s], ph ^ 1, p.err, abort_flag)) {
+                        uint8_t *A = stages + s * C::A_BYTES;
+                        const uint32_t bytes = (pg0 >= 0 ? 64 * DI : 0) + (pg1 >= 0 ? 64 * DI : 0);
+                        if (bytes) {
+                            mbar_expect_tx(&full[s], bytes);
+                            if (pg0 >= 0) tma_load_2d(A, &kmap, &full[s], 0, pg0 * 64);
+                            if (pg1 >= 0) tma_load_2d(A + 64 * DI, &kmap, &full[s], 0, pg1 * 64);
+                        } else {
+                            mbar_arrive(&full[s]);
+                        }
+                        ++issued;
+                    } else {
+                        ok = false;
+                    }
+                }
+                if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+                    ok = false;
+                    break;
+                }
+            }
+            tq = tq_n, p0 = p0_n, p1 = p1_n;
         }
         // never leave a copy in flight behind
-        for (int i = issued - 1; i >= 0 && i >= issued - C::STAGES; --i)
-            mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1, p.err, nullptr);
+        if (lane == 0) {
+            for (int i = issued - 1; i >= 0 && i >= issued - C::STAGES; --i)
+                mbar_wait(&full[i % C::STAGES], (i / C::STAGES) & 1, p.err, nullptr);
+            if (qo >= 0) mbar_wait(&qfull[qo & 1], (qo >> 1) & 1, p.err, nullptr);
+        }
     } else if (warp == 1 && lane == 0 && n > 0) {
         // ---------------- MMA issuer ----------------
         constexpr uint32_t ID = idesc(0, 0, 0, 0, NH, 128);
+        int t = locate(tstart, T, lo);
+        int j = static_cast<int>(lo - tstart[t]);
+        int qo = -1, tprev = -1;
         for (int i = 0; i < n; ++i) {
+            if (t != tprev) {  // the query changes: release the old heads, wait for the new
+                if (qo >= 0) mma_commit(&qempty[qo & 1]);
+                tprev = t;
+                ++qo;
+                if (!mbar_wait(&qfull[qo & 1], (qo >> 1) & 1, p.err, abort_flag)) break;
+            }
             const int s = i % C::STAGES;
             const uint32_t ph = (i / C::STAGES) & 1;
             const int a = i % C::ACC;
@@ -227,8 +291,8 @@ __global__ void __launch_bounds__(192, 1)
             if (!mbar_wait(&full[s], ph, p.err, abort_flag)) break;
             if (!mbar_wait(&tempty[a], aph ^ 1, p.err, abort_flag)) break;
             tc_fence_after();
-            const uint32_t A = smem_u32(stages + s * C::STAGE_BYTES);
-            const uint32_t B = A + C::A_BYTES;
+            const uint32_t A = smem_u32(stages + s * C::A_BYTES);
+            const uint32_t B = smem_u32(qbuf + (qo & 1) * C::B_BYTES);
             const uint32_t d = tmem + a * NH;
 #pragma unroll
             for (int k = 0; k < DI / 32; ++k)
@@ -236,51 +300,58 @@ __global__ void __launch_bounds__(192, 1)
                          k > 0);
             mma_commit(&empty[s]);
             mma_commit(&tfull[a]);
+            if (++j == tstart[t + 1] - tstart[t]) {
+                j = 0;
+                do { ++t; } while (t < T && tstart[t + 1] == tstart[t]);
+            }
         }
         mma_commit(drain);
         mbar_wait(drain, 0, p.err, nullptr);
     } else if (warp >= 2 && n > 0) {
-        // ---------------- epilogue ----------------
+        // ---------------- epilogue: warpgroup eg takes tiles i with i % EPI_GROUPS == eg ----------------
+        const int eg = (warp - 2) >> 2;
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
         int t = locate(tstart, T, lo);
         int j = static_cast<int>(lo - tstart[t]);
-        QInfo qi = query_info(t, p.q_seq, p.q_pos, p.pg, p.max_len, p.err);
+        int tw = -1;  // query whose w is in registers
+        QInfo qi{0, -1};
         float wr[NH];
-#pragma unroll
-        for (int h = 0; h < NH; ++h) wr[h] = h < p.HI ? p.w[(int64_t)t * p.HI + h] : 0.f;
         for (int i = 0; i < n; ++i) {
-            const int a = i % C::ACC;
-            const uint32_t aph = (i / C::ACC) & 1;
-            if (!mbar_wait(&tfull[a], aph, p.err, abort_flag)) break;
-            tc_fence_after();
-            uint32_t r[NH];
-            const uint32_t ta = tmem + a * NH + lane_off;
-            if constexpr (NH == 16) {
-                tmem_ld16(ta, r);
-            } else {
-#pragma unroll
-                for (int c = 0; c < NH / 32; ++c) tmem_ld32(ta + 32 * c, r + 32 * c);
-            }
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[a]);
-            float sc = 0.f;
-#pragma unroll
-            for (int h = 0; h < NH; ++h)
-                if (h < p.HI) sc = fmaf(wr[h], fmaxf(__uint_as_float(r[h]), 0.f), sc);
-            const int spos = j * 128 + row;
-            if (spos <= qi.last) p.scores[(int64_t)t * p.ld + spos] = sc;
-            if (++j == tstart[t + 1] - tstart[t]) {
-                j = 0;
-                do { ++t; } while (t < T && tstart[t + 1] == tstart[t]);
-                if (t < T) {
+            if (i % C::EPI_GROUPS == eg) {
+                if (t != tw) {
+                    tw = t;
                     qi = query_info(t, p.q_seq, p.q_pos, p.pg, p.max_len, p.err);
 #pragma unroll
                     for (int h = 0; h < NH; ++h) wr[h] = h < p.HI ? p.w[(int64_t)t * p.HI + h] : 0.f;
                 }
+                const int a = i % C::ACC;
+                const uint32_t aph = (i / C::ACC) & 1;
+                if (!mbar_wait(&tfull[a], aph, p.err, abort_flag)) break;
+                tc_fence_after();
+                uint32_t r[NH];
+                const uint32_t ta = tmem + a * NH + lane_off;
+                if constexpr (NH == 16) {
+                    tmem_ld16(ta, r);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < NH / 32; ++c) tmem_ld32(ta + 32 * c, r + 32 * c);
+                }
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[a]);
+                float sc = 0.f;
+#pragma unroll
+                for (int h = 0; h < NH; ++h)
+                    if (h < p.HI) sc = fmaf(wr[h], fmaxf(__uint_as_float(r[h]), 0.f), sc);
+                const int spos = j * 128 + row;
+                if (spos <= qi.last) p.scores[(int64_t)t * p.ld + spos] = sc;
+            }
+            if (++j == tstart[t + 1] - tstart[t]) {
+                j = 0;
+                do { ++t; } while (t < T && tstart[t + 1] == tstart[t]);
             }
         }
     }
@@ -303,7 +374,8 @@ struct PreCfg {
     static constexpr int A_BYTES = 128 * DI;
     static constexpr int B_BYTES = N * DI;
     static constexpr int ASTAGES = DI == 128 ? 6 : 10;
-    static constexpr int TMEM_COLS = 512;
+    static constexpr int TMEM_COLS = 512;  // two 256-column accumulators, one per epilogue warpgroup
+    static constexpr int THREADS = 64 + 256;
     static constexpr uint32_t SWZ = DI == 128 ? SWZ_128B : SWZ_64B;
     static constexpr uint32_t SBO = 8 * DI;
     static constexpr int BAR_BYTES = 8 * (2 * ASTAGES + 4 + 4 + 1);
@@ -345,7 +417,7 @@ __device__ __forceinline__ int group_of(int r, int c, int grid, int ngroups) {
 }
 
 template <int DI, int HI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(PreCfg<DI, HI>::THREADS, 1)
     indexer_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                            const IdxParams p) {
     using C = PreCfg<DI, HI>;
@@ -396,7 +468,10 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ---------------- producer (warp loads tables, lane 0 issues) ----------------
+        // ---------------- producer ----------------
+        // The warp loads the group table and, per run, looks up the pages of
+        // 32 key tiles at a time (one per lane, the next window in flight while
+        // lane 0 issues the current one).
         int ac = 0, issued_a = 0, gi = 0;
         bool ok = true;
         for (int r = 0; ok; ++r, ++gi) {
@@ -404,42 +479,63 @@ __global__ void __launch_bounds__(192, 1)
             if (g < 0) break;
             load_group_tbl(tbl_p, g, G, p, false, lane, 32);
             __syncwarp();
+            const int bst = gi & 1;
             if (lane == 0) {
-                const int bst = gi & 1;
                 if (!mbar_wait(&bempty[bst], ((gi >> 1) & 1) ^ 1, p.err, abort_flag)) ok = false;
                 if (ok) {
                     mbar_expect_tx(&bfull[bst], C::B_BYTES);
                     tma_load_2d(Bbuf + bst * C::B_BYTES, &qmap, &bfull[bst], 0, g * G * HI);
                 }
-                for (int u = 0; ok && u < G;) {
-                    int u1, b;
-                    const int nt = next_run(tbl_p, G, u, &u1, &b);
-                    int mx = -1;
-                    for (int v = u; v < u1; ++v) mx = max(mx, tbl_p[v].y);
-                    for (int kt = 0; kt < nt; ++kt) {
-                        const int s = ac % C::ASTAGES;
-                        if (!mbar_wait(&aempty[s], ((ac / C::ASTAGES) & 1) ^ 1, p.err, abort_flag)) {
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            for (int u = 0; ok && u < G;) {
+                int u1, b;
+                const int nt = next_run(tbl_p, G, u, &u1, &b);
+                int mx = -1;
+                for (int v = u; v < u1; ++v) mx = max(mx, tbl_p[v].y);
+                auto lookup = [&](int kt, int &q0, int &q1) {
+                    q0 = -1, q1 = -1;
+                    if (kt < nt) {
+                        q0 = page_of(p.pg, b, 2 * kt, p.err);
+                        q1 = (2 * kt + 1) * 64 <= mx ? page_of(p.pg, b, 2 * kt + 1, p.err) : -1;
+                    }
+                };
+                int q0, q1;
+                lookup(lane, q0, q1);
+                for (int base = 0; ok && base < nt; base += 32) {
+                    int q0n, q1n;
+                    lookup(base + 32 + lane, q0n, q1n);
+                    const int cnt = min(32, nt - base);
+                    for (int k = 0; k < cnt; ++k) {
+                        const int pg0 = __shfl_sync(0xffffffffu, q0, k);
+                        const int pg1 = __shfl_sync(0xffffffffu, q1, k);
+                        if (lane == 0) {
+                            const int s = ac % C::ASTAGES;
+                            if (mbar_wait(&aempty[s], ((ac / C::ASTAGES) & 1) ^ 1, p.err, abort_flag)) {
+                                uint8_t *A = Abuf + s * C::A_BYTES;
+                                const uint32_t bytes = (pg0 >= 0 ? 64 * DI : 0) + (pg1 >= 0 ? 64 * DI : 0);
+                                if (bytes) {
+                                    mbar_expect_tx(&afull[s], bytes);
+                                    if (pg0 >= 0) tma_load_2d(A, &kmap, &afull[s], 0, pg0 * 64);
+                                    if (pg1 >= 0) tma_load_2d(A + 64 * DI, &kmap, &afull[s], 0, pg1 * 64);
+                                } else {
+                                    mbar_arrive(&afull[s]);
+                                }
+                                ++ac;
+                                issued_a = ac;
+                            } else {
+                                ok = false;
+                            }
+                        }
+                        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
                             ok = false;
                             break;
                         }
-                        uint8_t *A = Abuf + s * C::A_BYTES;
-                        const int pg0 = page_of(p.pg, b, 2 * kt, p.err);
-                        const int pg1 = (2 * kt + 1) * 64 <= mx ? page_of(p.pg, b, 2 * kt + 1, p.err) : -1;
-                        const uint32_t bytes = (pg0 >= 0 ? 64 * DI : 0) + (pg1 >= 0 ? 64 * DI : 0);
-                        if (bytes) {
-                            mbar_expect_tx(&afull[s], bytes);
-                            if (pg0 >= 0) tma_load_2d(A, &kmap, &afull[s], 0, pg0 * 64);
-                            if (pg1 >= 0) tma_load_2d(A + 64 * DI, &kmap, &afull[s], 0, pg1 * 64);
-                        } else {
-                            mbar_arrive(&afull[s]);
-                        }
-                        ++ac;
-                        issued_a = ac;
                     }
-                    u = u1;
+                    q0 = q0n, q1 = q1n;
                 }
+                u = u1;
             }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         }
         if (lane == 0) {
             for (int i = issued_a - 1; i >= 0 && i >= issued_a - C::ASTAGES; --i)
@@ -493,8 +589,10 @@ __global__ void __launch_bounds__(192, 1)
             mbar_wait(drain, 0, p.err, nullptr);
         }
     } else {
-        // ---------------- epilogue (warps 2..5) ----------------
-        const int et = threadIdx.x - 64;  // 0..127
+        // ---------------- epilogue: two warpgroups (warps 2..5, 6..9) ----------------
+        // Tile tc lives in TMEM buffer tc % 2 and is reduced by warpgroup tc % 2.
+        const int et = threadIdx.x - 64;  // 0..255
+        const int eg = et >> 7;
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
@@ -503,18 +601,19 @@ __global__ void __launch_bounds__(192, 1)
         for (int r = 0; ok; ++r) {
             const int g = group_of(r, cta, grid, ngroups);
             if (g < 0) break;
-            named_bar_sync(1, 128);
-            load_group_tbl(tbl_e, g, G, p, true, et, 128);
-            for (int i = et; i < C::N; i += 128) {
+            named_bar_sync(1, 256);
+            load_group_tbl(tbl_e, g, G, p, true, et, 256);
+            for (int i = et; i < C::N; i += 256) {
                 const int t = g * G + i / HI;
                 wbuf[i] = t < p.T ? p.w[(int64_t)t * HI + (i % HI)] : 0.f;
             }
-            named_bar_sync(1, 128);
+            named_bar_sync(1, 256);
             for (int u = 0; ok && u < G;) {
                 int u1, b;
                 const int nt = next_run(tbl_e, G, u, &u1, &b);
-                for (int kt = 0; kt < nt; ++kt) {
+                for (int kt = 0; kt < nt; ++kt, ++tc) {
                     const int a = tc & 1;
+                    if (a != eg) continue;
                     if (!mbar_wait(&tfull[a], (tc >> 1) & 1, p.err, abort_flag)) {
                         ok = false;
                         break;
@@ -557,11 +656,11 @@ __global__ void __launch_bounds__(192, 1)
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&tempty[a]);
-                    ++tc;
                 }
                 u = u1;
             }
-            ok = !*abort_flag;
+            // the epilogue warpgroups leave the group loop together
+            ok = !named_bar_or(1, 256, !ok || *abort_flag);
         }
     }
     tc_fence_before();
@@ -577,7 +676,7 @@ dsa_status run_decode(const CUtensorMap &km, const CUtensorMap &qm, const IdxPar
     using C = DecCfg<DI, NH>;
     auto fn = indexer_decode_kernel<DI, NH>;
     if (!ensure_smem(reinterpret_cast<const void *>(fn), C::SMEM)) return DSA_ERR_CUDA;
-    fn<<<grid, 192, C::SMEM, st>>>(km, qm, p);
+    fn<<<grid, C::THREADS, C::SMEM, st>>>(km, qm, p);
     return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -587,7 +686,7 @@ dsa_status run_prefill(const CUtensorMap &km, const CUtensorMap &qm, const IdxPa
     using C = PreCfg<DI, HI>;
     auto fn = indexer_prefill_kernel<DI, HI>;
     if (!ensure_smem(reinterpret_cast<const void *>(fn), C::SMEM)) return DSA_ERR_CUDA;
-    fn<<<grid, 192, C::SMEM, st>>>(km, qm, p);
+    fn<<<grid, C::THREADS, C::SMEM, st>>>(km, qm, p);
     return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -611,7 +710,8 @@ dsa_status launch_indexer(const IndexerArgs &a, cudaStream_t st) {
                           swz))
             return DSA_ERR_INVALID_ARG;
         const int64_t tiles_bound = (int64_t)a.T * ((a.max_len + 127) / 128);
-        const int grid = (int)(tiles_bound < dev->sm_count ? tiles_bound : dev->sm_count);
+        const int64_t slots = (int64_t)dev->sm_count * DecCfg<128, 32>::CTAS_PER_SM;
+        const int grid = (int)(tiles_bound < slots ? tiles_bound : slots);
         if (grid <= 0) return DSA_OK;
         if (a.DI == 128) {
             if (NH == 16) return run_decode<128, 16>(km, qm, p, grid, st);

@@ -7,12 +7,13 @@
 // lower position and -0.0 equals +0.0.  The kept positions are written in
 // ascending order, padded with -1.
 //
-// Exact radix select on order-preserving 32-bit keys: three digit passes
-// (11, 11 and 10 bits) find the K-th largest key tau and the number `need`
+// Exact radix select on order-preserving 32-bit keys: digit passes find the
+// K-th largest key tau and the number `need`
 // of keys equal to tau that are kept; a stable compaction in position order
 // then takes every key > tau and the first `need` keys == tau.
-//   * rows up to SMALL_CAP keys: one CTA per row, keys resident in shared
-//     memory, histograms in shared memory;
+//   * rows whose slice fits in shared memory: one thread-block cluster per
+//     row (8 CTAs when rows are few, 1 when they are many), four 8-bit passes,
+//     histograms merged through distributed shared memory;
 //   * longer rows: CHUNK-key slices per CTA, per-row global histograms, the
 //     last CTA of a pass (atomic ticket, no waiting) picks the digit; then a
 //     count pass and an offset-and-write pass.
@@ -24,8 +25,6 @@
 namespace dsa {
 namespace {
 
-constexpr int SMALL_THREADS = 1024;
-constexpr int SMALL_CAP = 49152;  // keys resident in shared memory (192 KB)
 constexpr int CHUNK = 4096;       // keys per CTA on the multi-CTA path
 constexpr int MULTI_THREADS = 256;
 constexpr int HBINS = 2048;
@@ -148,46 +147,207 @@ __device__ void compact(KeyAt key_at, int s0, int s1, uint32_t tau, uint32_t nee
 }
 
 // ---------------------------------------------------------------------------
-// one CTA per row, keys in shared memory
+// One thread-block cluster per row (CL CTAs; CL = 1 for many short rows).
+// Each CTA holds its contiguous slice of the row as keys in shared memory
+// (RESIDENT) or re-reads it from global memory (L2) every pass.  The row's
+// key range is found first; 8-bit radix passes then run below the bits all
+// keys share, with warp-private histograms summed across the cluster through
+// distributed shared memory after one hardware cluster barrier per pass.  Compaction: warp ballots in position order, one
+// cluster exchange of per-CTA counts for the offsets.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(SMALL_THREADS, 1) topk_small_kernel(const TopkArgs a, uint32_t *err) {
-    extern __shared__ uint32_t sm[];
-    uint32_t *hist = sm;                   // [HBINS]
-    uint32_t *scan = hist + HBINS;         // [SMALL_THREADS]
-    uint32_t *wsum = scan + SMALL_THREADS;  // [32]
-    uint32_t *misc = wsum + 32;            // [8]
-    uint32_t *keys = misc + 8;             // [max_row_len]
-    const int r = blockIdx.x;
-    const int n = row_length(a, r, err);
+constexpr int CT_THREADS = 1024;
+constexpr int CT_WARPS = CT_THREADS / 32;
+constexpr int CT_FIXED_SMEM = (CT_WARPS * 256 + 2 * 256 + 256 + CT_WARPS * 4 + 16) * 4;
+
+template <int CL, bool RESIDENT>
+__global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkArgs a, uint32_t *err) {
+    extern __shared__ __align__(16) uint32_t sm[];
+    uint32_t *whist = sm;                      // [32][256] warp-private histograms
+    uint32_t *chist = whist + CT_WARPS * 256;  // [2][256] this CTA's histogram (read by the cluster)
+    uint32_t *tot = chist + 2 * 256;           // [256] the cluster's histogram
+    uint32_t *wcnt = tot + 256;                // [32][4] per-warp (gt, eq) counts and prefixes
+    uint32_t *misc = wcnt + CT_WARPS * 4;      // [16] (8..11: key range)
+    uint32_t *keys = misc + 16;                // [slice] (RESIDENT)
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t crank = CL > 1 ? cluster_ctarank() : 0;
+    const int r = blockIdx.x / CL;
+    const int n = row_length(a, r, crank == 0 ? err : nullptr);
     int32_t *out = a.idx + (int64_t)r * a.K;
-    if (n <= a.K) {
-        for (int j = threadIdx.x; j < a.K; j += SMALL_THREADS) out[j] = j < n ? j : -1;
+    if (n <= a.K) {  // uniform across the cluster: every CTA returns here
+        const int per = (a.K + CL - 1) / CL;
+        for (int j = crank * per + tid; j < min(a.K, (int)(crank + 1) * per); j += CT_THREADS) out[j] = j < n ? j : -1;
         return;
     }
-    const float *row = a.scores + (int64_t)r * a.ld;
-    for (int s = threadIdx.x; s < n; s += SMALL_THREADS) keys[s] = score_key(row[s]);
-    uint32_t prefix = 0, remaining = (uint32_t)a.K;
-    for (int ps = 0; ps < 3; ++ps) {
-        const int shift = kPass[ps].shift, bits = kPass[ps].bits;
-        const int nb = 1 << bits;
-        for (int i = threadIdx.x; i < nb; i += SMALL_THREADS) hist[i] = 0;
-        __syncthreads();
-        const int hs = shift + bits;
-        for (int s = threadIdx.x; s < n; s += SMALL_THREADS) {
-            const uint32_t k = keys[s];
-            if (hs == 32 || (k >> hs) == prefix) atomicAdd(&hist[(k >> shift) & (nb - 1)], 1u);
+    const int len = (n + CL - 1) / CL;
+    const int s0 = crank * len;
+    const int m = max(0, min(n, s0 + len) - s0);
+    const float *row = a.scores + (int64_t)r * a.ld + s0;
+    auto key_at = [&](int i) -> uint32_t { return RESIDENT ? keys[i] : score_key(__ldg(row + i)); };
+    // ---- the row's key range: bits above the highest bit where min and max
+    // differ are shared by every key, so the digit passes start below them.
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int i = tid; i < m; i += CT_THREADS) {
+        const uint32_t k = score_key(row[i]);
+        if (RESIDENT) keys[i] = k;
+        kmin = min(kmin, k);
+        kmax = max(kmax, k);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    }
+    if (lane == 0) {
+        wcnt[warp * 4 + 0] = kmin;
+        wcnt[warp * 4 + 1] = kmax;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t a0 = wcnt[lane * 4 + 0], a1 = wcnt[lane * 4 + 1];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            a0 = min(a0, __shfl_xor_sync(0xffffffffu, a0, o));
+            a1 = max(a1, __shfl_xor_sync(0xffffffffu, a1, o));
+        }
+        if (lane == 0) {
+            misc[8] = a0;
+            misc[9] = a1;
+        }
+    }
+    if (CL > 1) cluster_sync(); else __syncthreads();
+    if (tid == 0) {
+        uint32_t g0 = misc[8], g1 = misc[9];
+        for (int q = 0; q < CL; ++q) {
+            if (q == (int)crank) continue;
+            g0 = min(g0, ld_dsmem_u32(misc + 8, q));
+            g1 = max(g1, ld_dsmem_u32(misc + 9, q));
+        }
+        misc[10] = g0;
+        misc[11] = g1;
+    }
+    __syncthreads();
+    const uint32_t gmin = misc[10], gmax = misc[11];
+    int bits = gmin == gmax ? 0 : 32 - __clz(gmin ^ gmax);
+    uint32_t prefix = bits >= 32 ? 0u : (gmax >> bits), remaining = (uint32_t)a.K;
+    for (int ps = 0; bits > 0; ++ps) {
+        const int d = bits < 8 ? bits : 8;
+        const int shift = bits - d;
+        const int hs = shift + d;
+        uint32_t *wh = whist + warp * 256;
+        for (int b = lane; b < 256; b += 32) wh[b] = 0;
+        __syncthreads();  // keys loaded; every warp's histogram cleared
+        for (int i = tid; i < m; i += CT_THREADS) {
+            const uint32_t k = key_at(i);
+            if (hs >= 32 || (k >> hs) == prefix) atomicAdd(&wh[(k >> shift) & 255u], 1u);
         }
         __syncthreads();
-        int2 *res = reinterpret_cast<int2 *>(misc);
-        if (threadIdx.x == 0) *res = make_int2(0, 0);
+        uint32_t *ch = chist + (ps & 1) * 256;
+        if (tid < 256) {
+            uint32_t c = 0;
+#pragma unroll 8
+            for (int w = 0; w < CT_WARPS; ++w) c += whist[w * 256 + tid];
+            ch[tid] = c;
+        }
+        if (CL > 1) cluster_sync(); else __syncthreads();
+        if (tid < 256) {
+            uint32_t c = 0;
+            for (int q = 0; q < CL; ++q) c += CL > 1 ? ld_dsmem_u32(ch + tid, q) : ch[tid];
+            tot[tid] = c;
+        }
         __syncthreads();
-        pick_bin<SMALL_THREADS>(hist, nb, remaining, scan, res);
-        prefix = (prefix << bits) | (uint32_t)res->x;
-        remaining -= (uint32_t)res->y;
+        if (warp == 0) {
+            // lane l owns bins 255-8l .. 248-8l (from the top)
+            uint32_t v[8], sum = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                v[i] = tot[255 - 8 * lane - i];
+                sum += v[i];
+            }
+            uint32_t incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += x;
+            }
+            const uint32_t excl = incl - sum;
+            if (excl < remaining && remaining <= incl) {
+                uint32_t above = excl;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (above + v[i] >= remaining) {
+                        misc[0] = 255 - 8 * lane - i;
+                        misc[1] = above;
+                        break;
+                    }
+                    above += v[i];
+                }
+            }
+        }
         __syncthreads();
+        prefix = (prefix << d) | misc[0];
+        remaining -= misc[1];
+        bits = shift;
     }
-    compact<SMALL_THREADS>([&](int s) { return keys[s]; }, 0, n, prefix, remaining, 0, 0, out, a.K, wsum, misc + 4,
-                          err);
+    const uint32_t tau = prefix, need = remaining;
+
+    // ---- compaction: warp w owns positions [w*per, (w+1)*per) of the slice
+    const int per = (((m + CT_WARPS - 1) / CT_WARPS) + 31) & ~31;
+    const int w0 = warp * per, w1 = min(m, w0 + per);
+    uint32_t g = 0, e = 0;
+    for (int i0 = w0; i0 < w1; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t k = i < w1 ? key_at(i) : 0u;
+        g += __popc(__ballot_sync(0xffffffffu, i < w1 && k > tau));
+        e += __popc(__ballot_sync(0xffffffffu, i < w1 && k == tau));
+    }
+    if (lane == 0) {
+        wcnt[warp * 4 + 0] = g;
+        wcnt[warp * 4 + 1] = e;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t gv = wcnt[lane * 4 + 0], ev = wcnt[lane * 4 + 1];
+        uint32_t gi = gv, ei = ev;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t xg = __shfl_up_sync(0xffffffffu, gi, o), xe = __shfl_up_sync(0xffffffffu, ei, o);
+            if (lane >= o) gi += xg, ei += xe;
+        }
+        wcnt[lane * 4 + 2] = gi - gv;
+        wcnt[lane * 4 + 3] = ei - ev;
+        if (lane == 31) {
+            misc[4] = gi;  // this CTA's totals, read by later CTAs of the cluster
+            misc[5] = ei;
+        }
+    }
+    if (CL > 1) cluster_sync(); else __syncthreads();
+    if (tid == 0) {
+        uint32_t gb = 0, eb = 0;
+        for (int q = 0; q < (int)crank; ++q) {
+            gb += ld_dsmem_u32(misc + 4, q);
+            eb += ld_dsmem_u32(misc + 5, q);
+        }
+        misc[6] = gb;
+        misc[7] = eb;
+    }
+    __syncthreads();
+    uint32_t gcur = misc[6] + wcnt[warp * 4 + 2], ecur = misc[7] + wcnt[warp * 4 + 3];
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int i0 = w0; i0 < w1; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t k = i < w1 ? key_at(i) : 0u;
+        const bool gt = i < w1 && k > tau, eq = i < w1 && k == tau;
+        const uint32_t gm = __ballot_sync(0xffffffffu, gt), em = __ballot_sync(0xffffffffu, eq);
+        const uint32_t mg = gcur + __popc(gm & lt), me = ecur + __popc(em & lt);
+        if (gt || (eq && me < need)) {
+            const uint32_t slot = mg + min(me, need);
+            if (slot < (uint32_t)a.K) out[slot] = s0 + i;
+            else record_error(err, DSA_DEVERR_SHAPE);
+        }
+        gcur += __popc(gm);
+        ecur += __popc(em);
+    }
+    if (CL > 1) cluster_sync();  // no CTA leaves while another may still read its shared memory
 }
 
 // ---------------------------------------------------------------------------
@@ -330,27 +490,68 @@ __global__ void __launch_bounds__(MULTI_THREADS) topk_write_kernel(const TopkArg
                            need, before[0], before[1], out, a.K, wsum, tot, err);
 }
 
+struct ClusterPlan {
+    int cl;         // CTAs per row (0: use the multi-launch path)
+    bool resident;  // slice kept in shared memory
+    int smem;
+};
+
+// Short rows are many (prefill): one CTA per row.  Few rows: 8 CTAs per row.
+// The slice must fit in shared memory; longer rows go to the multi-launch path.
+ClusterPlan cluster_plan(int R, int max_row_len, const DeviceInfo *dev) {
+    ClusterPlan cp{0, true, 0};
+    const int cl = (R >= dev->sm_count / 2) ? 1 : 8;
+    const int slice = (max_row_len + cl - 1) / cl;
+    const int smem = CT_FIXED_SMEM + slice * 4;
+    if (smem <= dev->max_smem_optin) cp = ClusterPlan{cl, true, smem};
+    return cp;
+}
+
+template <int CL, bool RES>
+dsa_status launch_cluster_t(const TopkArgs &a, int smem, cudaStream_t st, uint32_t *err) {
+    auto fn = topk_cluster_kernel<CL, RES>;
+    if (!ensure_smem(reinterpret_cast<const void *>(fn), smem)) return DSA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.R * CL);
+    cfg.blockDim = dim3(CT_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fn, a, err) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status launch_cluster(const TopkArgs &a, const ClusterPlan &cp, cudaStream_t st, uint32_t *err) {
+    if (cp.cl == 1) return launch_cluster_t<1, true>(a, cp.smem, st, err);
+    return launch_cluster_t<8, true>(a, cp.smem, st, err);
+}
+
 }  // namespace
 
 size_t topk_workspace_bytes(int32_t R, int32_t K, int32_t max_row_len) {
     (void)K;
-    if (max_row_len <= SMALL_CAP) return 0;
+    const DeviceInfo *dev = current_device();
+    if (dev && cluster_plan(R, max_row_len, dev).cl > 0) return 0;
     const int nch = (max_row_len + CHUNK - 1) / CHUNK;
     return align_up(multi_zero_bytes(R) + (size_t)R * nch * 2 * 4, 256);
 }
 
-int topk_kernel_launches(int32_t max_row_len) { return max_row_len <= SMALL_CAP ? 1 : 5; }
+int topk_kernel_launches(int32_t R, int32_t max_row_len) {
+    const DeviceInfo *dev = current_device();
+    return (dev && cluster_plan(R, max_row_len, dev).cl > 0) ? 1 : 5;
+}
 
 dsa_status launch_topk(const TopkArgs &a, cudaStream_t st) {
     const DeviceInfo *dev = current_device();
     if (!dev) return DSA_ERR_CUDA;
     if (a.R == 0) return DSA_OK;
-    if (a.max_row_len <= SMALL_CAP) {
-        const int smem = (HBINS + SMALL_THREADS + 32 + 8) * 4 + a.max_row_len * 4;
-        if (!ensure_smem(reinterpret_cast<const void *>(topk_small_kernel), smem)) return DSA_ERR_CUDA;
-        topk_small_kernel<<<a.R, SMALL_THREADS, smem, st>>>(a, dev->err);
-        return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
-    }
+    const ClusterPlan cp = cluster_plan(a.R, a.max_row_len, dev);
+    if (cp.cl > 0) return launch_cluster(a, cp, st, dev->err);
     const size_t need = topk_workspace_bytes(a.R, a.K, a.max_row_len);
     if (a.ws == nullptr || a.ws_bytes < need) return DSA_ERR_WORKSPACE;
     MultiWs m = carve_multi(a.ws, a.R, a.max_row_len);

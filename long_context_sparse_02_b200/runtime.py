@@ -53,6 +53,10 @@ class LayerOnDevice:
         _lib.layer_forward(self.args, self.ws)
         return self.out
 
+    def forward_profiled(self, events):
+        _lib.layer_forward_profiled(self.args, self.ws, events)
+        return self.out
+
     @property
     def scores(self) -> torch.Tensor:
         """The fp32 scores the last forward left at the head of the workspace."""
