@@ -18,6 +18,7 @@
 //     last CTA of a pass (atomic ticket, no waiting) picks the digit; then a
 //     count pass and an offset-and-write pass.
 #include <mutex>
+#include <vector>
 
 #include "dsa_device.cuh"
 #include "dsa_internal.h"
@@ -148,26 +149,266 @@ __device__ void compact(KeyAt key_at, int s0, int s1, uint32_t tau, uint32_t nee
 
 // ---------------------------------------------------------------------------
 // One thread-block cluster per row (CL CTAs; CL = 1 for many short rows).
-// Each CTA holds its contiguous slice of the row as keys in shared memory
-// (RESIDENT) or re-reads it from global memory (L2) every pass.  The row's
-// key range is found first; 8-bit radix passes then run below the bits all
-// keys share, with warp-private histograms summed across the cluster through
-// distributed shared memory after one hardware cluster barrier per pass.  Compaction: warp ballots in position order, one
-// cluster exchange of per-CTA counts for the offsets.
+// Each CTA holds its contiguous slice of the row (raw fp32 scores) in shared
+// memory.
+//
+//   1. load the slice (16-byte loads); the row's key range [min, max] over
+//      the cluster (barrier 1);
+//   2. a histogram of LBINS equal-width bins over [min, max] in score space.
+//      The bin of a score x is floor((x - min) * LBINS / (max - min)) in
+//      fp32 with every rounding monotone, so the bins split the row into
+//      consecutive key intervals.  Each CTA bins its slice, then adds its
+//      counts into the CTA that owns each bin (LBINS / CL bins per CTA;
+//      barrier 2);
+//   3. every CTA reads the totals (one 8-byte remote load per thread) and
+//      finds the bin b holding the K-th largest key.  One sweep of the slice
+//      lists, per warp and in position order, the positions whose bin is
+//      >= b, and collects the keys of bin b (barrier 3).  Every key in a bin
+//      above b is kept; an exact select on the cluster's keys of bin b (few
+//      unless the row is degenerate) gives the threshold key tau and how
+//      many keys equal to tau are kept;
+//   4. stable compaction of the listed positions (the whole slice when a
+//      warp's list overflows) in position order.
+// Rows whose bin b holds more than CAND_CAP keys (heavy ties, an outlier
+// that squeezes the rest into one bin) or whose range is not finite fall
+// back to 8-bit radix passes over the whole slice.  Counts and candidates
+// move through distributed shared memory.
 // ---------------------------------------------------------------------------
 constexpr int CT_THREADS = 1024;
 constexpr int CT_WARPS = CT_THREADS / 32;
-constexpr int CT_FIXED_SMEM = (CT_WARPS * 256 + 2 * 256 + 256 + CT_WARPS * 4 + 16) * 4;
+constexpr int LBINS = 2048;
+constexpr int CAND_CAP = 4096;  // keys of the threshold bin, whole cluster
+constexpr int WCAP = 128;       // listed positions per warp
+constexpr int RANK_MAX = 128;   // at most this many candidates: select by counting ranks
+// shared memory, in 32-bit words
+constexpr int CT_W_WORDS = CT_WARPS * 256;  // radix warp histograms | candidate lists
+constexpr int OWN_WORDS = LBINS / 2;        // bins owned by one CTA (CL >= 2)
+constexpr int CT_FIXED_WORDS =
+    CT_W_WORDS + LBINS + OWN_WORDS + CT_WARPS * WCAP + 2 * 256 + 256 + CT_WARPS * 4 + 64;
+constexpr int CT_FIXED_SMEM = CT_FIXED_WORDS * 4;
+static_assert(CT_W_WORDS >= 2 * CAND_CAP, "candidate lists alias the radix histograms");
+static_assert(CT_FIXED_WORDS % 4 == 0, "the slice starts 16-byte aligned");
+static_assert(LBINS == 2 * CT_THREADS, "two bins per thread");
+// misc words: 0,1 digit/bin pick; 2 candidate counter; 3 keys in bin b (cluster);
+// 4,5 CTA totals (radix path) / tau, need; 6,7 offsets; 8,9 CTA key range;
+// 10,11 row key range; 12,13 sums; 20,21 this CTA's keys above b / in b;
+// 22 list overflow; 24,25 above-b keys / bin-b keys of earlier CTAs;
+// 32..47 bin-b keys of earlier CTAs, per CTA rank
 
-template <int CL, bool RESIDENT>
+__device__ __forceinline__ int linear_bin(float x, float lo, float scale) {
+    const float y = __fmul_rn(__fsub_rn(x, lo), scale);
+    return min(LBINS - 1, __float2int_rz(y));
+}
+__device__ __forceinline__ float key_score(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+__device__ __forceinline__ uint32_t dsmem_addr(const void *local, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+    return remote;
+}
+__device__ __forceinline__ void dsmem_red_add(uint32_t remote, uint32_t v) {
+    asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint2 dsmem_ld_v2(uint32_t remote) {
+    uint2 v;
+    asm volatile("ld.shared::cluster.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(remote) : "memory");
+    return v;
+}
+
+// Block-wide (CT_THREADS) inclusive scan; ws holds CT_WARPS words.
+__device__ __forceinline__ uint32_t ct_incl_scan(uint32_t v, uint32_t *ws) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) ws[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t t = ws[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
+        }
+        ws[lane] = t;
+    }
+    __syncthreads();
+    return x + (warp > 0 ? ws[warp - 1] : 0u);
+}
+
+// Block-wide sums of two counters; ws holds 2 * CT_WARPS words, out 2 words.
+__device__ __forceinline__ void ct_sum2(uint32_t a, uint32_t b, uint32_t *ws, uint32_t *out) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        b += __shfl_xor_sync(0xffffffffu, b, o);
+    }
+    if (lane == 0) {
+        ws[2 * warp] = a;
+        ws[2 * warp + 1] = b;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t x = ws[2 * lane], y = ws[2 * lane + 1];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            x += __shfl_xor_sync(0xffffffffu, x, o);
+            y += __shfl_xor_sync(0xffffffffu, y, o);
+        }
+        if (lane == 0) {
+            out[0] = x;
+            out[1] = y;
+        }
+    }
+    __syncthreads();
+}
+
+// Warp 0: from a 256-bin digit histogram (tot), the digit holding the
+// remaining-th largest key and the count of keys in higher digits -> res[0..1].
+__device__ __forceinline__ void pick_digit256(const uint32_t *tot, uint32_t remaining, uint32_t *res) {
+    const int lane = threadIdx.x & 31;
+    uint32_t v[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {  // lane l owns digits 255-8l .. 248-8l (from the top)
+        v[i] = tot[255 - 8 * lane - i];
+        sum += v[i];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += x;
+    }
+    const uint32_t excl = incl - sum;
+    if (excl < remaining && remaining <= incl) {
+        uint32_t above = excl;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (above + v[i] >= remaining) {
+                res[0] = 255 - 8 * lane - i;
+                res[1] = above;
+                break;
+            }
+            above += v[i];
+        }
+    }
+}
+
+// barrier.cluster in two halves: arrive after the last read of another CTA's
+// shared memory, wait before leaving (a CTA's shared memory must outlive
+// every remote access to it).
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
+template <int CL>
+__device__ __forceinline__ void ct_cluster_or_block_sync() {
+    if (CL > 1) cluster_sync();
+    else __syncthreads();
+}
+
+// Exact select among C keys (block-wide): the rem-th largest key -> res[0]
+// and how many keys equal to it are among the rem largest -> res[1].
+__device__ void select_among(const uint32_t *cand, int C, uint32_t rem, uint32_t *hist, uint32_t *wcnt,
+                             uint32_t *res) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (C <= RANK_MAX) {
+        // rank of key j in the order (key descending, index ascending)
+        if (tid < C) {
+            const uint32_t kj = cand[tid];
+            uint32_t g = 0, e = 0;
+            for (int i = 0; i < C; ++i) {
+                const uint32_t ki = cand[i];
+                g += ki > kj;
+                e += (ki == kj) & (i < tid);
+            }
+            if (g + e == rem - 1) {
+                res[0] = kj;
+                res[1] = rem - g;
+            }
+        }
+        __syncthreads();
+        return;
+    }
+    uint32_t cmn = 0xFFFFFFFFu, cmx = 0u;
+    for (int j = tid; j < C; j += CT_THREADS) {
+        cmn = min(cmn, cand[j]);
+        cmx = max(cmx, cand[j]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        cmn = min(cmn, __shfl_xor_sync(0xffffffffu, cmn, o));
+        cmx = max(cmx, __shfl_xor_sync(0xffffffffu, cmx, o));
+    }
+    if (lane == 0) {
+        wcnt[warp * 4 + 2] = cmn;
+        wcnt[warp * 4 + 3] = cmx;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t a0 = wcnt[lane * 4 + 2], a1 = wcnt[lane * 4 + 3];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            a0 = min(a0, __shfl_xor_sync(0xffffffffu, a0, o));
+            a1 = max(a1, __shfl_xor_sync(0xffffffffu, a1, o));
+        }
+        if (lane == 0) {
+            res[2] = a0;
+            res[3] = a1;
+        }
+    }
+    __syncthreads();
+    const uint32_t c0 = res[2], c1 = res[3];
+    int bits = c0 == c1 ? 0 : 32 - __clz(c0 ^ c1);
+    uint32_t prefix = bits >= 32 ? 0u : (c1 >> bits), remaining = rem;
+    while (bits > 0) {
+        const int d = bits < 8 ? bits : 8;
+        const int shift = bits - d, hs = shift + d;
+        if (tid < 256) hist[tid] = 0;
+        __syncthreads();
+        for (int j = tid; j < C; j += CT_THREADS) {
+            const uint32_t k = cand[j];
+            if (hs >= 32 || (k >> hs) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+        }
+        __syncthreads();
+        if (warp == 0) pick_digit256(hist, remaining, res);
+        __syncthreads();
+        prefix = (prefix << d) | res[0];
+        remaining -= res[1];
+        bits = shift;
+        __syncthreads();  // res[0..1] read by every thread before the next pick
+    }
+    __syncthreads();
+    if (tid == 0) {
+        res[0] = prefix;
+        res[1] = remaining;
+    }
+    __syncthreads();
+}
+
+template <int CL>
 __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkArgs a, uint32_t *err) {
     extern __shared__ __align__(16) uint32_t sm[];
-    uint32_t *whist = sm;                      // [32][256] warp-private histograms
-    uint32_t *chist = whist + CT_WARPS * 256;  // [2][256] this CTA's histogram (read by the cluster)
-    uint32_t *tot = chist + 2 * 256;           // [256] the cluster's histogram
-    uint32_t *wcnt = tot + 256;                // [32][4] per-warp (gt, eq) counts and prefixes
-    uint32_t *misc = wcnt + CT_WARPS * 4;      // [16] (8..11: key range)
-    uint32_t *keys = misc + 16;                // [slice] (RESIDENT)
+    uint32_t *whist = sm;                  // radix path: [32][256] warp-private histograms
+    uint32_t *cand_local = sm;             // binned path: this CTA's keys of bin b (read by the cluster)
+    uint32_t *cand_all = sm + CAND_CAP;    // binned path: the cluster's keys of bin b, CTA order
+    uint32_t *lhist = sm + CT_W_WORDS;     // [LBINS] this CTA's linear histogram
+    uint32_t *own = lhist + LBINS;         // [LBINS / CL] cluster totals of the bins this CTA owns
+    uint32_t *wlist = own + OWN_WORDS;     // [32][WCAP] per-warp listed positions
+    uint32_t *chist = wlist + CT_WARPS * WCAP;  // [2][256] radix path: this CTA's digit histogram
+    uint32_t *lcnt = chist;                // [32] binned path: listed positions per warp
+    uint32_t *tot = chist + 2 * 256;       // [256] digit histogram
+    uint32_t *wcnt = tot + 256;            // [32][4] per-warp scratch
+    uint32_t *misc = wcnt + CT_WARPS * 4;  // [64] scalars (see above)
+    float *xs = reinterpret_cast<float *>(misc + 64);  // [slice] the scores
+    constexpr int W = LBINS / CL;          // bins owned per CTA
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t crank = CL > 1 ? cluster_ctarank() : 0;
     const int r = blockIdx.x / CL;
@@ -178,19 +419,54 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
         for (int j = crank * per + tid; j < min(a.K, (int)(crank + 1) * per); j += CT_THREADS) out[j] = j < n ? j : -1;
         return;
     }
-    const int len = (n + CL - 1) / CL;
-    const int s0 = crank * len;
-    const int m = max(0, min(n, s0 + len) - s0);
+    const int len = ((n + CL - 1) / CL + 3) & ~3;  // slices start 4 keys apart
+    const int s0 = min(n, (int)crank * len);
+    const int m = min(n, s0 + len) - s0;
     const float *row = a.scores + (int64_t)r * a.ld + s0;
-    auto key_at = [&](int i) -> uint32_t { return RESIDENT ? keys[i] : score_key(__ldg(row + i)); };
-    // ---- the row's key range: bits above the highest bit where min and max
-    // differ are shared by every key, so the digit passes start below them.
+
+    // ---- 1. load the slice; its key range.  Histograms and counters are
+    // cleared here: barrier 1 orders that before any CTA adds into them.
+    for (int i = tid; i < LBINS; i += CT_THREADS) lhist[i] = 0;
+    if (CL > 1)
+        for (int i = tid; i < W; i += CT_THREADS) own[i] = 0;
+    if (tid == 0) misc[2] = 0;
     uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-    for (int i = tid; i < m; i += CT_THREADS) {
-        const uint32_t k = score_key(row[i]);
-        if (RESIDENT) keys[i] = k;
-        kmin = min(kmin, k);
-        kmax = max(kmax, k);
+    {
+        int done = 0;
+        if ((reinterpret_cast<uintptr_t>(row) & 15u) == 0) {
+            const int m4 = m >> 2;
+            const float4 *r4 = reinterpret_cast<const float4 *>(row);
+            float4 *x4 = reinterpret_cast<float4 *>(xs);
+            constexpr int U = 4;
+            for (int base = 0; base < m4; base += U * CT_THREADS) {
+                float4 v[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int i = base + u * CT_THREADS + tid;
+                    if (i < m4) v[u] = r4[i];
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int i = base + u * CT_THREADS + tid;
+                    if (i < m4) {
+                        x4[i] = v[u];
+                        const uint32_t k0 = score_key(v[u].x), k1 = score_key(v[u].y), k2 = score_key(v[u].z),
+                                       k3 = score_key(v[u].w);
+                        kmin = min(kmin, min(min(k0, k1), min(k2, k3)));
+                        kmax = max(kmax, max(max(k0, k1), max(k2, k3)));
+                    }
+                }
+            }
+            done = m4 * 4;
+        }
+#pragma unroll 4
+        for (int i = done + tid; i < m; i += CT_THREADS) {
+            const float x = row[i];
+            xs[i] = x;
+            const uint32_t k = score_key(x);
+            kmin = min(kmin, k);
+            kmax = max(kmax, k);
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -214,91 +490,238 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
             misc[9] = a1;
         }
     }
-    if (CL > 1) cluster_sync(); else __syncthreads();
-    if (tid == 0) {
-        uint32_t g0 = misc[8], g1 = misc[9];
-        for (int q = 0; q < CL; ++q) {
-            if (q == (int)crank) continue;
-            g0 = min(g0, ld_dsmem_u32(misc + 8, q));
-            g1 = max(g1, ld_dsmem_u32(misc + 9, q));
+    ct_cluster_or_block_sync<CL>();  // cluster barrier 1: every CTA's range is published
+    if (warp == 0) {
+        uint32_t g0 = 0xFFFFFFFFu, g1 = 0u;
+        if (lane < CL) {
+            g0 = CL > 1 ? ld_dsmem_u32(misc + 8, lane) : misc[8];
+            g1 = CL > 1 ? ld_dsmem_u32(misc + 9, lane) : misc[9];
         }
-        misc[10] = g0;
-        misc[11] = g1;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            g0 = min(g0, __shfl_xor_sync(0xffffffffu, g0, o));
+            g1 = max(g1, __shfl_xor_sync(0xffffffffu, g1, o));
+        }
+        if (lane == 0) {
+            misc[10] = g0;
+            misc[11] = g1;
+        }
     }
     __syncthreads();
     const uint32_t gmin = misc[10], gmax = misc[11];
-    int bits = gmin == gmax ? 0 : 32 - __clz(gmin ^ gmax);
-    uint32_t prefix = bits >= 32 ? 0u : (gmax >> bits), remaining = (uint32_t)a.K;
-    for (int ps = 0; bits > 0; ++ps) {
-        const int d = bits < 8 ? bits : 8;
-        const int shift = bits - d;
-        const int hs = shift + d;
-        uint32_t *wh = whist + warp * 256;
-        for (int b = lane; b < 256; b += 32) wh[b] = 0;
-        __syncthreads();  // keys loaded; every warp's histogram cleared
-        for (int i = tid; i < m; i += CT_THREADS) {
-            const uint32_t k = key_at(i);
-            if (hs >= 32 || (k >> hs) == prefix) atomicAdd(&wh[(k >> shift) & 255u], 1u);
+
+    if (gmin == gmax) {  // every key equal: the first K positions (uniform across the cluster)
+        if (CL > 1) cluster_arrive();  // the range reads above were the last remote reads
+        for (int i = tid; i < m && s0 + i < a.K; i += CT_THREADS) out[s0 + i] = s0 + i;
+        if (CL > 1) cluster_wait();
+        return;
+    }
+
+    uint32_t tau = 0, need = 0, gt_before = 0, eq_before = 0;
+    bool binned = false, use_list = false;  // binned: uniform across the cluster
+    const float lo = key_score(gmin), hi = key_score(gmax);
+    const float width = __fsub_rn(hi, lo);
+    const float scale = __fdiv_rn((float)LBINS, width);
+    if (isfinite(lo) && isfinite(hi) && isfinite(width) && width > 0.f && isfinite(scale)) {
+        // ---- 2. linear histogram over [lo, hi]; counts into the owning CTAs
+        for (int i = tid; i < m; i += CT_THREADS) atomicAdd(&lhist[linear_bin(xs[i], lo, scale)], 1u);
+        __syncthreads();
+        if (CL > 1) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int bin = tid + h * CT_THREADS;
+                const uint32_t v = lhist[bin];
+                if (v) dsmem_red_add(dsmem_addr(own + bin % W, bin / W), v);
+            }
+        }
+        ct_cluster_or_block_sync<CL>();  // cluster barrier 2: every total is complete
+        // ---- 3. the bin of the K-th largest key (thread t: bins LBINS-1-2t, LBINS-2-2t)
+        const int hb0 = LBINS - 1 - 2 * tid, hb1 = hb0 - 1;
+        uint2 t2;
+        if (CL > 1) t2 = dsmem_ld_v2(dsmem_addr(own + hb1 % W, hb1 / W));
+        else t2 = make_uint2(lhist[hb1], lhist[hb0]);
+        const uint32_t v0 = t2.y, v1 = t2.x;
+        const uint32_t incl = ct_incl_scan(v0 + v1, wcnt);
+        const uint32_t excl = incl - v0 - v1, Ku = (uint32_t)a.K;
+        if (excl < Ku && Ku <= incl) {
+            const bool first = excl + v0 >= Ku;
+            misc[0] = first ? hb0 : hb1;
+            misc[1] = first ? excl : excl + v0;
+            misc[3] = first ? v0 : v1;
         }
         __syncthreads();
-        uint32_t *ch = chist + (ps & 1) * 256;
-        if (tid < 256) {
-            uint32_t c = 0;
-#pragma unroll 8
-            for (int w = 0; w < CT_WARPS; ++w) c += whist[w * 256 + tid];
-            ch[tid] = c;
-        }
-        if (CL > 1) cluster_sync(); else __syncthreads();
-        if (tid < 256) {
-            uint32_t c = 0;
-            for (int q = 0; q < CL; ++q) c += CL > 1 ? ld_dsmem_u32(ch + tid, q) : ch[tid];
-            tot[tid] = c;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            // lane l owns bins 255-8l .. 248-8l (from the top)
-            uint32_t v[8], sum = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                v[i] = tot[255 - 8 * lane - i];
-                sum += v[i];
-            }
-            uint32_t incl = sum;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += x;
-            }
-            const uint32_t excl = incl - sum;
-            if (excl < remaining && remaining <= incl) {
-                uint32_t above = excl;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    if (above + v[i] >= remaining) {
-                        misc[0] = 255 - 8 * lane - i;
-                        misc[1] = above;
-                        break;
-                    }
-                    above += v[i];
+        const int b = (int)misc[0];
+        const uint32_t above = misc[1], C = misc[3];
+        if (C <= (uint32_t)CAND_CAP) {
+            binned = true;
+            // one sweep: per-warp lists of positions with bin >= b (position
+            // order) and this CTA's keys of bin b
+            const int per = (((m + CT_WARPS - 1) / CT_WARPS) + 31) & ~31;
+            const int w0 = warp * per, w1 = min(m, w0 + per);
+            uint32_t cnt = 0;
+            uint32_t *wl = wlist + warp * WCAP;
+            const uint32_t lt = (1u << lane) - 1u;
+            for (int i0 = w0; i0 < w1; i0 += 32) {
+                const int i = i0 + lane;
+                const float x = i < w1 ? xs[i] : 0.f;
+                const int bn = i < w1 ? linear_bin(x, lo, scale) : -1;
+                const uint32_t sel = __ballot_sync(0xffffffffu, bn >= b);
+                const uint32_t inb = __ballot_sync(0xffffffffu, bn == b);
+                if (bn >= b) {
+                    const uint32_t slot = cnt + __popc(sel & lt);
+                    if (slot < (uint32_t)WCAP) wl[slot] = (uint32_t)i;
+                }
+                cnt += __popc(sel);
+                if (inb) {
+                    uint32_t base = 0;
+                    if (lane == 0) base = atomicAdd(&misc[2], (uint32_t)__popc(inb));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    if (bn == b) cand_local[base + __popc(inb & lt)] = score_key(x);
                 }
             }
+            if (lane == 0) lcnt[warp] = cnt;
+            __syncthreads();
+            if (warp == 0) {
+                const uint32_t c = lcnt[lane];
+                uint32_t s = c;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                const bool ovf = __any_sync(0xffffffffu, c > (uint32_t)WCAP);
+                if (lane == 0) {
+                    misc[20] = s - lhist[b];  // keys above b in this CTA
+                    misc[21] = lhist[b];      // keys in b in this CTA
+                    misc[22] = ovf;
+                }
+            }
+            ct_cluster_or_block_sync<CL>();  // cluster barrier 3: every candidate list is complete
+            use_list = misc[22] == 0;
+            if (warp == 0) {
+                uint32_t hq = 0, cq = 0;
+                if (lane < CL) {
+                    hq = CL > 1 ? ld_dsmem_u32(misc + 20, lane) : misc[20];
+                    cq = CL > 1 ? ld_dsmem_u32(misc + 21, lane) : misc[21];
+                }
+                uint32_t hx = hq, cx = cq;  // inclusive prefix over CTA ranks
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t y0 = __shfl_up_sync(0xffffffffu, hx, o), y1 = __shfl_up_sync(0xffffffffu, cx, o);
+                    if (lane >= o) hx += y0, cx += y1;
+                }
+                if (lane < CL) misc[32 + lane] = cx - cq;  // bin-b keys of earlier CTAs
+                if (lane == (int)crank) {
+                    misc[24] = hx - hq;
+                    misc[25] = cx - cq;
+                }
+            }
+            __syncthreads();
+            const uint32_t *cand = cand_local;
+            if (CL > 1) {
+                for (int j = tid; j < (int)C; j += CT_THREADS) {
+                    int q = 0;
+                    while (q < CL - 1 && (uint32_t)j >= misc[32 + q + 1]) ++q;
+                    cand_all[j] = ld_dsmem_u32(cand_local + (j - misc[32 + q]), q);
+                }
+                cluster_arrive();  // no more reads of other CTAs' shared memory
+                cand = cand_all;
+                __syncthreads();
+            }
+            select_among(cand, (int)C, Ku - above, tot, wcnt, misc + 4);
+            tau = misc[4];
+            need = misc[5];
+            const uint32_t hi_before = misc[24], c_before = misc[25];
+            uint32_t g = 0, e = 0;
+            for (int j = tid; j < (int)c_before; j += CT_THREADS) {
+                g += cand[j] > tau;
+                e += cand[j] == tau;
+            }
+            ct_sum2(g, e, wcnt, misc + 12);
+            gt_before = hi_before + misc[12];
+            eq_before = misc[13];
+        }
+    }
+
+    if (!binned) {
+        // ---- fallback: 8-bit radix passes over the whole slice
+        int bits = 32 - __clz(gmin ^ gmax);
+        uint32_t prefix = bits >= 32 ? 0u : (gmax >> bits), remaining = (uint32_t)a.K;
+        for (int ps = 0; bits > 0; ++ps) {
+            const int d = bits < 8 ? bits : 8;
+            const int shift = bits - d;
+            const int hs = shift + d;
+            uint32_t *wh = whist + warp * 256;
+            for (int b = lane; b < 256; b += 32) wh[b] = 0;
+            __syncthreads();  // every warp's histogram cleared
+            for (int i = tid; i < m; i += CT_THREADS) {
+                const uint32_t k = score_key(xs[i]);
+                if (hs >= 32 || (k >> hs) == prefix) atomicAdd(&wh[(k >> shift) & 255u], 1u);
+            }
+            __syncthreads();
+            uint32_t *ch = chist + (ps & 1) * 256;
+            if (tid < 256) {
+                uint32_t c = 0;
+#pragma unroll 8
+                for (int w = 0; w < CT_WARPS; ++w) c += whist[w * 256 + tid];
+                ch[tid] = c;
+            }
+            ct_cluster_or_block_sync<CL>();
+            if (tid < 256) {
+                uint32_t c = 0;
+                for (int q = 0; q < CL; ++q) c += CL > 1 ? ld_dsmem_u32(ch + tid, q) : ch[tid];
+                tot[tid] = c;
+            }
+            __syncthreads();
+            if (warp == 0) pick_digit256(tot, remaining, misc);
+            __syncthreads();
+            prefix = (prefix << d) | misc[0];
+            remaining -= misc[1];
+            bits = shift;
+        }
+        tau = prefix;
+        need = remaining;
+        // this CTA's counts, then the cluster's earlier CTAs' totals
+        uint32_t g = 0, e = 0;
+        for (int i = tid; i < m; i += CT_THREADS) {
+            const uint32_t k = score_key(xs[i]);
+            g += k > tau;
+            e += k == tau;
+        }
+        ct_sum2(g, e, wcnt, misc + 4);
+        ct_cluster_or_block_sync<CL>();
+        if (warp == 0) {
+            uint32_t gb = 0, eb = 0;
+            if (lane < (int)crank) {
+                gb = ld_dsmem_u32(misc + 4, lane);
+                eb = ld_dsmem_u32(misc + 5, lane);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                gb += __shfl_xor_sync(0xffffffffu, gb, o);
+                eb += __shfl_xor_sync(0xffffffffu, eb, o);
+            }
+            if (lane == 0) {
+                misc[6] = gb;
+                misc[7] = eb;
+            }
         }
         __syncthreads();
-        prefix = (prefix << d) | misc[0];
-        remaining -= misc[1];
-        bits = shift;
+        gt_before = misc[6];
+        eq_before = misc[7];
+        if (CL > 1) cluster_arrive();
     }
-    const uint32_t tau = prefix, need = remaining;
 
-    // ---- compaction: warp w owns positions [w*per, (w+1)*per) of the slice
+    // ---- 4. compaction in position order: warp w walks its listed positions
+    // (or all of [w*per, (w+1)*per) of the slice)
     const int per = (((m + CT_WARPS - 1) / CT_WARPS) + 31) & ~31;
-    const int w0 = warp * per, w1 = min(m, w0 + per);
+    const int w0 = warp * per;
+    const int wn = use_list ? (int)lcnt[warp] : max(0, min(m, w0 + per) - w0);
+    const uint32_t *wl = wlist + warp * WCAP;
+    auto pos_at = [&](int j) -> int { return use_list ? (int)wl[j] : w0 + j; };
     uint32_t g = 0, e = 0;
-    for (int i0 = w0; i0 < w1; i0 += 32) {
-        const int i = i0 + lane;
-        const uint32_t k = i < w1 ? key_at(i) : 0u;
-        g += __popc(__ballot_sync(0xffffffffu, i < w1 && k > tau));
-        e += __popc(__ballot_sync(0xffffffffu, i < w1 && k == tau));
+    for (int j0 = 0; j0 < wn; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t k = j < wn ? score_key(xs[pos_at(j)]) : 0u;
+        g += __popc(__ballot_sync(0xffffffffu, j < wn && k > tau));
+        e += __popc(__ballot_sync(0xffffffffu, j < wn && k == tau));
     }
     if (lane == 0) {
         wcnt[warp * 4 + 0] = g;
@@ -315,28 +738,15 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
         }
         wcnt[lane * 4 + 2] = gi - gv;
         wcnt[lane * 4 + 3] = ei - ev;
-        if (lane == 31) {
-            misc[4] = gi;  // this CTA's totals, read by later CTAs of the cluster
-            misc[5] = ei;
-        }
-    }
-    if (CL > 1) cluster_sync(); else __syncthreads();
-    if (tid == 0) {
-        uint32_t gb = 0, eb = 0;
-        for (int q = 0; q < (int)crank; ++q) {
-            gb += ld_dsmem_u32(misc + 4, q);
-            eb += ld_dsmem_u32(misc + 5, q);
-        }
-        misc[6] = gb;
-        misc[7] = eb;
     }
     __syncthreads();
-    uint32_t gcur = misc[6] + wcnt[warp * 4 + 2], ecur = misc[7] + wcnt[warp * 4 + 3];
+    uint32_t gcur = gt_before + wcnt[warp * 4 + 2], ecur = eq_before + wcnt[warp * 4 + 3];
     const uint32_t lt = (1u << lane) - 1u;
-    for (int i0 = w0; i0 < w1; i0 += 32) {
-        const int i = i0 + lane;
-        const uint32_t k = i < w1 ? key_at(i) : 0u;
-        const bool gt = i < w1 && k > tau, eq = i < w1 && k == tau;
+    for (int j0 = 0; j0 < wn; j0 += 32) {
+        const int j = j0 + lane;
+        const int i = j < wn ? pos_at(j) : 0;
+        const uint32_t k = j < wn ? score_key(xs[i]) : 0u;
+        const bool gt = j < wn && k > tau, eq = j < wn && k == tau;
         const uint32_t gm = __ballot_sync(0xffffffffu, gt), em = __ballot_sync(0xffffffffu, eq);
         const uint32_t mg = gcur + __popc(gm & lt), me = ecur + __popc(em & lt);
         if (gt || (eq && me < need)) {
@@ -347,7 +757,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
         gcur += __popc(gm);
         ecur += __popc(em);
     }
-    if (CL > 1) cluster_sync();  // no CTA leaves while another may still read its shared memory
+    if (CL > 1) cluster_wait();  // no CTA leaves while another may still read its shared memory
 }
 
 // ---------------------------------------------------------------------------
@@ -491,44 +901,86 @@ __global__ void __launch_bounds__(MULTI_THREADS) topk_write_kernel(const TopkArg
 }
 
 struct ClusterPlan {
-    int cl;         // CTAs per row (0: use the multi-launch path)
-    bool resident;  // slice kept in shared memory
+    int cl;  // CTAs per row (0: use the multi-launch path)
     int smem;
 };
 
-// Short rows are many (prefill): one CTA per row.  Few rows: 8 CTAs per row.
-// The slice must fit in shared memory; longer rows go to the multi-launch path.
-ClusterPlan cluster_plan(int R, int max_row_len, const DeviceInfo *dev) {
-    ClusterPlan cp{0, true, 0};
-    const int cl = (R >= dev->sm_count / 2) ? 1 : 8;
-    const int slice = (max_row_len + cl - 1) / cl;
-    const int smem = CT_FIXED_SMEM + slice * 4;
-    if (smem <= dev->max_smem_optin) cp = ClusterPlan{cl, true, smem};
-    return cp;
+int cluster_smem(int max_row_len, int cl) {
+    const int slice = ((max_row_len + cl - 1) / cl + 3) & ~3;
+    return CT_FIXED_SMEM + slice * 4;
 }
 
-template <int CL, bool RES>
-dsa_status launch_cluster_t(const TopkArgs &a, int smem, cudaStream_t st, uint32_t *err) {
-    auto fn = topk_cluster_kernel<CL, RES>;
-    if (!ensure_smem(reinterpret_cast<const void *>(fn), smem)) return DSA_ERR_CUDA;
+template <int CL>
+cudaLaunchConfig_t cluster_cfg(int R, int smem, cudaStream_t st, cudaLaunchAttribute *attr) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.R * CL);
+    cfg.gridDim = dim3(R * CL);
     cfg.blockDim = dim3(CT_THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = CL;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    return cfg;
+}
+
+// How many 16-CTA clusters of this kernel the device runs at once (0 when it
+// cannot), cached per device and shared-memory size.
+int max_active_clusters16(const DeviceInfo *dev, int smem) {
+    static std::mutex mu;
+    static std::vector<std::pair<std::pair<int, int>, int>> memo;
+    std::lock_guard<std::mutex> lk(mu);
+    for (auto &e : memo)
+        if (e.first.first == dev->device && e.first.second == smem) return e.second;
+    int num = 0;
+    auto fn = topk_cluster_kernel<16>;
+    if (ensure_smem(reinterpret_cast<const void *>(fn), smem) &&
+        cudaFuncSetAttribute(reinterpret_cast<const void *>(fn), cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+            cudaSuccess) {
+        cudaLaunchAttribute attr[1];
+        cudaLaunchConfig_t cfg = cluster_cfg<16>(1, smem, 0, attr);
+        if (cudaOccupancyMaxActiveClusters(&num, fn, &cfg) != cudaSuccess) num = 0;
+    }
+    cudaGetLastError();
+    memo.push_back({{dev->device, smem}, num});
+    return num;
+}
+
+// Few rows: 16 CTAs per row when every row's cluster runs at once, else 8.
+// Many rows (prefill): one CTA per row.  A row whose slice does not fit in
+// shared memory is split over more CTAs (up to 8); longer rows go to the
+// multi-launch path.
+ClusterPlan cluster_plan(int R, int max_row_len, const DeviceInfo *dev) {
+    if (R * 16 <= dev->sm_count) {
+        const int smem = cluster_smem(max_row_len, 16);
+        if (smem <= dev->max_smem_optin && max_active_clusters16(dev, smem) >= R) return ClusterPlan{16, smem};
+    }
+    for (int cl = (R >= dev->sm_count / 2) ? 1 : 8; cl <= 8; cl *= 2) {
+        const int smem = cluster_smem(max_row_len, cl);
+        if (smem <= dev->max_smem_optin) return ClusterPlan{cl, smem};
+    }
+    return ClusterPlan{0, 0};
+}
+
+template <int CL>
+dsa_status launch_cluster_t(const TopkArgs &a, int smem, cudaStream_t st, uint32_t *err) {
+    auto fn = topk_cluster_kernel<CL>;
+    if (!ensure_smem(reinterpret_cast<const void *>(fn), smem)) return DSA_ERR_CUDA;
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = cluster_cfg<CL>(a.R, smem, st, attr);
     return cudaLaunchKernelEx(&cfg, fn, a, err) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 dsa_status launch_cluster(const TopkArgs &a, const ClusterPlan &cp, cudaStream_t st, uint32_t *err) {
-    if (cp.cl == 1) return launch_cluster_t<1, true>(a, cp.smem, st, err);
-    return launch_cluster_t<8, true>(a, cp.smem, st, err);
+    switch (cp.cl) {
+        case 1: return launch_cluster_t<1>(a, cp.smem, st, err);
+        case 2: return launch_cluster_t<2>(a, cp.smem, st, err);
+        case 4: return launch_cluster_t<4>(a, cp.smem, st, err);
+        case 8: return launch_cluster_t<8>(a, cp.smem, st, err);
+        default: return launch_cluster_t<16>(a, cp.smem, st, err);
+    }
 }
 
 }  // namespace

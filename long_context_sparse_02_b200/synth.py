@@ -223,7 +223,8 @@ def swa_case(seed: int, seq_lens, H: int = 64, D: int = 128, window: int = 128) 
 def score_rows(seed: int, R: int, n: int, kind: str = "normal") -> np.ndarray:
     """Synthetic score rows for exercising top-K alone.
     kind: 'normal' (N(0,1) fp32), 'ties' (few distinct values), 'zeros'
-    (+0/-0 mix), 'const' (all equal), 'dyadic' (multiples of 2^-14)."""
+    (+0/-0 mix), 'const' (all equal), 'dyadic' (multiples of 2^-14),
+    'outlier' (N(0,1) and one score of 1e30 per row)."""
     rng = np.random.default_rng(seed)
     if kind == "normal":
         return rng.standard_normal((R, n), dtype=np.float32)
@@ -238,4 +239,8 @@ def score_rows(seed: int, R: int, n: int, kind: str = "normal") -> np.ndarray:
         return np.full((R, n), 1.5, dtype=np.float32)
     if kind == "dyadic":
         return rng.integers(-(1 << 16), 1 << 16, size=(R, n)).astype(np.float32) * (2.0 ** -14)
+    if kind == "outlier":  # N(0,1) with one huge score per row
+        v = rng.standard_normal((R, n), dtype=np.float32)
+        v[np.arange(R), rng.integers(0, n, size=R)] = 1e30
+        return v
     raise ValueError(kind)

@@ -125,6 +125,8 @@ TOPK_CASES = [
     (9, 5000, 1, "dyadic"), (3, 49152, 2048, "ties"),
     (3, 70000, 2048, "normal"), (2, 131072, 2048, "dyadic"), (2, 90001, 2048, "ties"), (2, 60000, 17, "const"),
     (1, 300000, 2048, "zeros"),
+    (8, 131072, 2048, "normal"), (4, 4000, 2048, "outlier"), (2, 131072, 2048, "outlier"),
+    (80, 70000, 2048, "normal"), (76, 120000, 2048, "dyadic"),
 ]
 
 
