@@ -267,11 +267,20 @@ dsa_status layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes, dsa
     TopkArgs ta{lw.scores, ld, decode ? a->pg.seq_lens : a->q_pos,
                 decode ? (int32_t)ROWLEN_SEQ_LENS : (int32_t)ROWLEN_QPOS_PLUS_1,
                 a->T, a->K, a->max_len, lw.idx, lw.topk_ws, lw.topk_bytes};
+    ta.pdl = true;
+    if (decode) {  // the attention reads the kept rows next: start bringing them into L2
+        ta.pf_kv = static_cast<const uint8_t *>(static_cast<const void *>(a->kv_cache));
+        ta.pf_block_table = a->pg.block_table;
+        ta.pf_max_blocks = a->pg.max_blocks_per_seq;
+        ta.pf_num_pages = a->pg.num_pages;
+        ta.pf_row_bytes = a->Dqk * 2;
+    }
     s = launch_topk(ta, st);
     if (s != DSA_OK) return s;
     if (!mark(2)) return DSA_ERR_CUDA;
     AttnArgs aa{a->q, a->kv_cache, pg, decode ? nullptr : a->q_seq, lw.idx, a->K, a->gate, a->sm_scale, a->T, a->H,
                 a->Dqk, a->Dv, a->out, a->lse, lw.attn_ws, lw.attn_bytes};
+    aa.pdl = true;
     s = launch_attn(aa, st);
     if (s != DSA_OK) return s;
     return mark(3) ? DSA_OK : DSA_ERR_CUDA;

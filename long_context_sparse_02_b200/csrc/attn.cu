@@ -20,6 +20,8 @@
 //
 // Warps 0-3: softmax/epilogue (one TMEM lane quarter each, a thread per
 // head); warp 4: MMA issuer and TMEM owner; warps 5-8: gather producers.
+#include <utility>
+
 #include "dsa_device.cuh"
 #include "dsa_internal.h"
 
@@ -149,6 +151,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     }
     if (warp == 4) tmem_alloc(tmem_slot, C::TMEM_COLS);
     __syncthreads();
+    pdl_trigger();
+    pdl_wait();  // the selection comes from the previous kernel
     if (tok_ok)
         for (int g = row0 + threadIdx.x; g < row_end; g += ATT_THREADS)
             if (p.idx[(int64_t)t * p.K + g] >= 0) atomicMax(last_sh, g);
@@ -527,6 +531,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
             mbar_expect_tx(&q_full[kb], C::Q_STAGE);
             tma_load_2d(ring + kb * C::Q_STAGE, &qmap, &q_full[kb], kb * 64, t * p.H);
         }
+    pdl_trigger();
+    pdl_wait();  // the selection comes from the previous kernel
     if (threadIdx.x < DEC_NR) {  // resolve every selected row once, through the block table
         const int64_t rid = tok_ok ? latent_row(ap, b, L, t, row0 + threadIdx.x, row_end, true) : -1;
         rowid[threadIdx.x] = rid;
@@ -721,74 +727,74 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
     }
 }
 
-// One warp per (token, head, 256-wide slice of the value dims):
+// One thread per (token, head, 16-byte chunk of the value row):
 // out = sigmoid(g) * sum_s w_s o_s with w_s = l_s 2^(m_s - M) / sum l 2^(m - M).
-// The split partials are loaded eight at a time before they are summed.
-constexpr int CMB_SLICE = 256;
-__global__ void __launch_bounds__(256) attn_decode_combine_kernel(const DecAttnParams p, const uint16_t *gate,
-                                                                  uint16_t *out, float *lse) {
-    const int nsl = (p.Dv + CMB_SLICE - 1) / CMB_SLICE;
-    const int wid = blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (wid >= p.T * p.H * nsl) return;
-    const int sl = wid % nsl;
-    const int h = (wid / nsl) % p.H;
-    const int t = wid / (nsl * p.H);
+// Every load of a thread (split maxima and sums, gate, partial chunks) is
+// independent of the others and issued before any is used.
+constexpr int CMB_THREADS = 256;
+constexpr int CMB_BATCH = 8;  // splits in flight per thread
+__global__ void __launch_bounds__(CMB_THREADS) attn_decode_combine_kernel(const DecAttnParams p, const uint16_t *gate,
+                                                                          uint16_t *out, float *lse) {
+    pdl_wait();  // the partials come from the previous kernel
+    const int nch = p.Dv / 8;
+    const int64_t gid = (int64_t)blockIdx.x * CMB_THREADS + threadIdx.x;
+    if (gid >= (int64_t)p.T * p.H * nch) return;
+    const int c = (int)(gid % nch);
+    const int th = (int)(gid / nch);  // t * H + h
+    const int t = th / p.H, h = th % p.H;
     const int S = p.splits;
-    float ms = -INFINITY, ls = 0.f;
-    if (lane < S) {
-        const float *ml = p.part_ml + (((int64_t)t * S + lane) * p.H + h) * 2;
-        ms = ml[0];
-        ls = ml[1];
-    }
-    float M = ls > 0.f ? ms : -INFINITY;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float wl = ls > 0.f ? ls * exp2f(ms - M) : 0.f;
-    float wsum = wl;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-    const float g = __bfloat162float(__ushort_as_bfloat16(gate[(int64_t)t * p.H + h]));
-    const float scale = wsum > 0.f ? (1.f / (1.f + __expf(-g))) / wsum : 0.f;
-    const float coef = wl * scale;
-    const int d0 = sl * CMB_SLICE + lane * 8;
-    const bool live = d0 < p.Dv;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    const uint16_t *base = p.part_o + ((int64_t)t * S * p.H + h) * p.Dv + d0;
+    const float g = __bfloat162float(__ushort_as_bfloat16(gate[th]));
+    const uint16_t *base = p.part_o + ((int64_t)t * S * p.H + h) * p.Dv + c * 8;
+    const float2 *ml = reinterpret_cast<const float2 *>(p.part_ml) + (int64_t)t * S * p.H + h;
     const int64_t sstride = (int64_t)p.H * p.Dv;
-    for (int s0 = 0; s0 < S; s0 += 8) {
-        uint4 v[8];
+    float M = -INFINITY, W = 0.f;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    // running merge over batches of splits: acc and W are kept relative to M
+    for (int s0 = 0; s0 < S; s0 += CMB_BATCH) {
+        float2 v[CMB_BATCH];
+        uint4 o[CMB_BATCH];
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-            v[u] = (live && s0 + u < S) ? *reinterpret_cast<const uint4 *>(base + (s0 + u) * sstride)
-                                        : make_uint4(0, 0, 0, 0);
+        for (int u = 0; u < CMB_BATCH; ++u) {
+            const bool in = s0 + u < S;
+            v[u] = in ? ml[(int64_t)(s0 + u) * p.H] : make_float2(-INFINITY, 0.f);
+            o[u] = in ? *reinterpret_cast<const uint4 *>(base + (s0 + u) * sstride) : make_uint4(0, 0, 0, 0);
+        }
+        float Mb = M;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const float c = __shfl_sync(0xffffffffu, coef, (s0 + u) & 31);
-            const float cc = s0 + u < S ? c : 0.f;
-            const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        for (int u = 0; u < CMB_BATCH; ++u)
+            if (v[u].y > 0.f) Mb = fmaxf(Mb, v[u].x);
+        if (Mb == -INFINITY) continue;  // nothing selected so far
+        const float r = M == -INFINITY ? 0.f : exp2f(M - Mb);
+        W *= r;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] *= r;
+        M = Mb;
+#pragma unroll
+        for (int u = 0; u < CMB_BATCH; ++u) {
+            const float w = v[u].y > 0.f ? v[u].y * exp2f(v[u].x - M) : 0.f;
+            W += w;
+            const uint32_t w4[4] = {o[u].x, o[u].y, o[u].z, o[u].w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                acc[2 * i] = fmaf(cc, __uint_as_float(w4[i] << 16), acc[2 * i]);
-                acc[2 * i + 1] = fmaf(cc, __uint_as_float(w4[i] & 0xFFFF0000u), acc[2 * i + 1]);
+                acc[2 * i] = fmaf(w, __uint_as_float(w4[i] << 16), acc[2 * i]);
+                acc[2 * i + 1] = fmaf(w, __uint_as_float(w4[i] & 0xFFFF0000u), acc[2 * i + 1]);
             }
         }
     }
-    if (live) {
-        uint4 o;
-        o.x = pack_bf16(acc[0], acc[1]);
-        o.y = pack_bf16(acc[2], acc[3]);
-        o.z = pack_bf16(acc[4], acc[5]);
-        o.w = pack_bf16(acc[6], acc[7]);
-        *reinterpret_cast<uint4 *>(out + ((int64_t)t * p.H + h) * p.Dv + d0) = o;
-    }
-    if (sl == 0 && lane == 0 && lse)
-        lse[(int64_t)t * p.H + h] = wsum > 0.f ? (M + __log2f(wsum)) * 0.69314718055994531f : -INFINITY;
+    const float sc = W > 0.f ? (1.f / (1.f + __expf(-g))) / W : 0.f;
+    uint4 r;
+    r.x = pack_bf16(acc[0] * sc, acc[1] * sc);
+    r.y = pack_bf16(acc[2] * sc, acc[3] * sc);
+    r.z = pack_bf16(acc[4] * sc, acc[5] * sc);
+    r.w = pack_bf16(acc[6] * sc, acc[7] * sc);
+    *reinterpret_cast<uint4 *>(out + (int64_t)th * p.Dv + c * 8) = r;
+    if (c == 0 && lse) lse[th] = W > 0.f ? (M + __log2f(W)) * 0.69314718055994531f : -INFINITY;
 }
 
 // Merges split partials: out = sigmoid(g) * sum_s w_s o_s with
 // w_s = l_s 2^(m_s - M) / sum_s' l_s' 2^(m_s' - M).
 __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
+    pdl_wait();  // the partials come from the previous kernel
     const int t = blockIdx.x;
     const int h = blockIdx.y * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -849,18 +855,34 @@ Plan plan_for(int T, int K, int Dv, int sm_count) {
     return pl;
 }
 
+// Launches fn<<<grid, block, smem, st>>>(args...), as a programmatic
+// dependent of the previous kernel in the stream when pdl is set.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*fn)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t st, bool pdl,
+                     Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, fn, std::forward<Args>(args)...);
+}
+
 template <int DQK, int DVP>
-dsa_status run_attn(const CUtensorMap &qm, const AttnParams &p, cudaStream_t st) {
+dsa_status run_attn(const CUtensorMap &qm, const AttnParams &p, bool pdl, cudaStream_t st) {
     using C = AttnCfg<DQK, DVP>;
     auto fn = attn_kernel<DQK, DVP>;
     if (!ensure_smem(reinterpret_cast<const void *>(fn), C::SMEM)) return DSA_ERR_CUDA;
     dim3 grid(p.nparts * p.splits, p.T);
-    fn<<<grid, ATT_THREADS, C::SMEM, st>>>(qm, p);
-    if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+    if (launch_k(fn, grid, dim3(ATT_THREADS), C::SMEM, st, pdl, qm, p) != cudaSuccess) return DSA_ERR_CUDA;
     if (p.splits > 1) {
         dim3 cg(p.T, (p.H + 7) / 8);
-        attn_combine_kernel<<<cg, 256, 0, st>>>(p);
-        if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+        if (launch_k(attn_combine_kernel, cg, dim3(256), 0, st, pdl, p) != cudaSuccess) return DSA_ERR_CUDA;
     }
     return DSA_OK;
 }
@@ -896,15 +918,17 @@ int attn_kernel_launches(int32_t T, int32_t K, int32_t Dv) {
 
 template <int DQK, int DV>
 dsa_status run_attn_decode(const CUtensorMap &qm, const DecAttnParams &p, const uint16_t *gate, uint16_t *out,
-                           float *lse, cudaStream_t st) {
+                           float *lse, bool pdl, cudaStream_t st) {
     using C = DecAttnCfg<DQK, DV>;
     auto fn = attn_decode_kernel<DQK, DV>;
     if (!ensure_smem(reinterpret_cast<const void *>(fn), C::SMEM)) return DSA_ERR_CUDA;
-    fn<<<dim3(p.splits, p.T), DEC_THREADS, C::SMEM, st>>>(qm, p);
-    if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
-    const int warps = p.T * p.H * ((p.Dv + CMB_SLICE - 1) / CMB_SLICE);
-    attn_decode_combine_kernel<<<(warps + 7) / 8, 256, 0, st>>>(p, gate, out, lse);
-    return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+    if (launch_k(fn, dim3(p.splits, p.T), dim3(DEC_THREADS), C::SMEM, st, pdl, qm, p) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    const int64_t threads = (int64_t)p.T * p.H * (p.Dv / 8);
+    return launch_k(attn_decode_combine_kernel, dim3((unsigned)((threads + CMB_THREADS - 1) / CMB_THREADS)),
+                    dim3(CMB_THREADS), 0, st, pdl, p, gate, out, lse) == cudaSuccess
+               ? DSA_OK
+               : DSA_ERR_CUDA;
 }
 
 dsa_status launch_attn(const AttnArgs &a, cudaStream_t st) {
@@ -932,8 +956,8 @@ dsa_status launch_attn(const AttnArgs &a, cudaStream_t st) {
         if (!a.ws || a.ws_bytes < dec_ws_bytes(a.T, a.H, a.K, a.Dv)) return DSA_ERR_WORKSPACE;
         dp.part_o = static_cast<uint16_t *>(a.ws);
         dp.part_ml = reinterpret_cast<float *>(static_cast<uint8_t *>(a.ws) + align_up(rows * a.Dv * 2, 256));
-        if (a.Dqk == 576 && a.Dv == 512) return run_attn_decode<576, 512>(qm, dp, a.gate, a.out, a.lse, st);
-        if (a.Dqk == 64 && a.Dv == 64) return run_attn_decode<64, 64>(qm, dp, a.gate, a.out, a.lse, st);
+        if (a.Dqk == 576 && a.Dv == 512) return run_attn_decode<576, 512>(qm, dp, a.gate, a.out, a.lse, a.pdl, st);
+        if (a.Dqk == 64 && a.Dv == 64) return run_attn_decode<64, 64>(qm, dp, a.gate, a.out, a.lse, a.pdl, st);
         return DSA_ERR_UNSUPPORTED;
     }
     Plan pl = plan_for(a.T, a.K, a.Dv, dev->sm_count);
@@ -961,8 +985,8 @@ dsa_status launch_attn(const AttnArgs &a, cudaStream_t st) {
         p.part_o = static_cast<float *>(a.ws);
         p.part_ml = reinterpret_cast<float *>(static_cast<uint8_t *>(a.ws) + align_up(rows * a.Dv * 4, 256));
     }
-    if (a.Dqk == 576 && a.Dv == 512) return run_attn<576, 256>(qm, p, st);
-    if (a.Dqk == 64 && a.Dv == 64) return run_attn<64, 64>(qm, p, st);
+    if (a.Dqk == 576 && a.Dv == 512) return run_attn<576, 256>(qm, p, a.pdl, st);
+    if (a.Dqk == 64 && a.Dv == 64) return run_attn<64, 64>(qm, p, a.pdl, st);
     return DSA_ERR_UNSUPPORTED;
 }
 

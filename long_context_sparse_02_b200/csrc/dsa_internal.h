@@ -59,6 +59,12 @@ struct TopkArgs {
     int32_t *idx;
     void *ws;
     size_t ws_bytes;
+    // optional (decode rows, row r = sequence r): the latent cache rows of the
+    // kept positions are prefetched into L2 for the attention that follows
+    const uint8_t *pf_kv;  // NULL: no prefetch
+    const int32_t *pf_block_table;
+    int32_t pf_max_blocks, pf_num_pages, pf_row_bytes;
+    bool pdl;  // launched as a programmatic dependent of the previous kernel
 };
 size_t topk_workspace_bytes(int32_t R, int32_t K, int32_t max_row_len);
 int topk_kernel_launches(int32_t R, int32_t max_row_len);
@@ -80,6 +86,7 @@ struct AttnArgs {
     float *lse;
     void *ws;
     size_t ws_bytes;
+    bool pdl;  // launched as a programmatic dependent of the previous kernel
 };
 size_t attn_workspace_bytes(int32_t T, int32_t H, int32_t K, int32_t Dv);
 int attn_kernel_launches(int32_t T, int32_t K, int32_t Dv);

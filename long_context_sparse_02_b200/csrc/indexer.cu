@@ -194,6 +194,7 @@ __global__ void __launch_bounds__(DecCfg<DI, NH>::THREADS, DecCfg<DI, NH>::CTAS_
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_trigger();
     const uint32_t tmem = *tmem_slot;
     const int64_t total = tstart[T];
     const int64_t lo = total * blockIdx.x / gridDim.x;
@@ -465,6 +466,7 @@ __global__ void __launch_bounds__(PreCfg<DI, HI>::THREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_trigger();
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {

@@ -183,8 +183,9 @@ constexpr int RANK_MAX = 128;   // at most this many candidates: select by count
 // shared memory, in 32-bit words
 constexpr int CT_W_WORDS = CT_WARPS * 256;  // radix warp histograms | candidate lists
 constexpr int OWN_WORDS = LBINS / 2;        // bins owned by one CTA (CL >= 2)
+constexpr int PF_PAGES = 512;  // block-table entries staged for the L2 prefetch
 constexpr int CT_FIXED_WORDS =
-    CT_W_WORDS + LBINS + OWN_WORDS + CT_WARPS * WCAP + 2 * 256 + 256 + CT_WARPS * 4 + 64;
+    CT_W_WORDS + LBINS + OWN_WORDS + CT_WARPS * WCAP + 2 * 256 + 256 + CT_WARPS * 4 + 64 + PF_PAGES;
 constexpr int CT_FIXED_SMEM = CT_FIXED_WORDS * 4;
 static_assert(CT_W_WORDS >= 2 * CAND_CAP, "candidate lists alias the radix histograms");
 static_assert(CT_FIXED_WORDS % 4 == 0, "the slice starts 16-byte aligned");
@@ -201,20 +202,6 @@ __device__ __forceinline__ int linear_bin(float x, float lo, float scale) {
 }
 __device__ __forceinline__ float key_score(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
-}
-
-__device__ __forceinline__ uint32_t dsmem_addr(const void *local, uint32_t rank) {
-    uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-    return remote;
-}
-__device__ __forceinline__ void dsmem_red_add(uint32_t remote, uint32_t v) {
-    asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint2 dsmem_ld_v2(uint32_t remote) {
-    uint2 v;
-    asm volatile("ld.shared::cluster.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(remote) : "memory");
-    return v;
 }
 
 // Block-wide (CT_THREADS) inclusive scan; ws holds CT_WARPS words.
@@ -299,14 +286,6 @@ __device__ __forceinline__ void pick_digit256(const uint32_t *tot, uint32_t rema
         }
     }
 }
-
-// barrier.cluster in two halves: arrive after the last read of another CTA's
-// shared memory, wait before leaving (a CTA's shared memory must outlive
-// every remote access to it).
-__device__ __forceinline__ void cluster_arrive() {
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 template <int CL>
 __device__ __forceinline__ void ct_cluster_or_block_sync() {
@@ -407,7 +386,8 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
     uint32_t *tot = chist + 2 * 256;       // [256] digit histogram
     uint32_t *wcnt = tot + 256;            // [32][4] per-warp scratch
     uint32_t *misc = wcnt + CT_WARPS * 4;  // [64] scalars (see above)
-    float *xs = reinterpret_cast<float *>(misc + 64);  // [slice] the scores
+    int32_t *pf_pages = reinterpret_cast<int32_t *>(misc + 64);  // [PF_PAGES] cache pages of the slice
+    float *xs = reinterpret_cast<float *>(pf_pages + PF_PAGES);  // [slice] the scores
     constexpr int W = LBINS / CL;          // bins owned per CTA
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t crank = CL > 1 ? cluster_ctarank() : 0;
@@ -423,6 +403,17 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
     const int s0 = min(n, (int)crank * len);
     const int m = min(n, s0 + len) - s0;
     const float *row = a.scores + (int64_t)r * a.ld + s0;
+    pdl_trigger();
+    // block-table entries of the slice, for the L2 prefetch of kept rows
+    const int pf_page0 = s0 >> 6;
+    const bool pf = a.pf_kv != nullptr && m > 0 && ((s0 + m - 1) >> 6) - pf_page0 < PF_PAGES;
+    if (pf)
+        for (int i = tid; i <= ((s0 + m - 1) >> 6) - pf_page0; i += CT_THREADS) {
+            const int lp = pf_page0 + i;
+            const int pg = lp < a.pf_max_blocks ? a.pf_block_table[(int64_t)r * a.pf_max_blocks + lp] : -1;
+            pf_pages[i] = (pg >= 0 && pg < a.pf_num_pages) ? pg : -1;
+        }
+    pdl_wait();  // the scores come from the previous kernel
 
     // ---- 1. load the slice; its key range.  Histograms and counters are
     // cleared here: barrier 1 orders that before any CTA adds into them.
@@ -512,7 +503,13 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
 
     if (gmin == gmax) {  // every key equal: the first K positions (uniform across the cluster)
         if (CL > 1) cluster_arrive();  // the range reads above were the last remote reads
-        for (int i = tid; i < m && s0 + i < a.K; i += CT_THREADS) out[s0 + i] = s0 + i;
+        for (int i = tid; i < m && s0 + i < a.K; i += CT_THREADS) {
+            out[s0 + i] = s0 + i;
+            if (pf) {
+                const int pos = s0 + i, pg = pf_pages[(pos >> 6) - pf_page0];
+                if (pg >= 0) l2_prefetch(a.pf_kv + ((int64_t)pg * 64 + (pos & 63)) * a.pf_row_bytes, a.pf_row_bytes);
+            }
+        }
         if (CL > 1) cluster_wait();
         return;
     }
@@ -753,6 +750,10 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
             const uint32_t slot = mg + min(me, need);
             if (slot < (uint32_t)a.K) out[slot] = s0 + i;
             else record_error(err, DSA_DEVERR_SHAPE);
+            if (pf) {
+                const int pos = s0 + i, pg = pf_pages[(pos >> 6) - pf_page0];
+                if (pg >= 0) l2_prefetch(a.pf_kv + ((int64_t)pg * 64 + (pos & 63)) * a.pf_row_bytes, a.pf_row_bytes);
+            }
         }
         gcur += __popc(gm);
         ecur += __popc(em);
@@ -968,8 +969,13 @@ template <int CL>
 dsa_status launch_cluster_t(const TopkArgs &a, int smem, cudaStream_t st, uint32_t *err) {
     auto fn = topk_cluster_kernel<CL>;
     if (!ensure_smem(reinterpret_cast<const void *>(fn), smem)) return DSA_ERR_CUDA;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = cluster_cfg<CL>(a.R, smem, st, attr);
+    if (a.pdl) {
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.numAttrs = 2;
+    }
     return cudaLaunchKernelEx(&cfg, fn, a, err) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 

@@ -155,7 +155,10 @@ def test_topk_bit_exact(L, orc, R, n, K, kind):
     (576, 512, 128, 2048, [300, 9000], 4, True),
     (576, 512, 40, 256, [2000], 16, True),
     (576, 512, 128, 512, [600, 3000], 64, True),
-], ids=["tiny", "tiny_pad", "full_T3", "full_decode_split", "heads40", "prefill_T64"])
+    (576, 512, 128, 960, [5000], 2, False),
+    (576, 512, 128, 2560, [3000, 9000], 3, True),
+], ids=["tiny", "tiny_pad", "full_T3", "full_decode_split", "heads40", "prefill_T64", "ragged_K960",
+        "K2560_two_kernel"])
 def test_sparse_attn_within_tolerance(L, orc, Dqk, Dv, H, K, seq_lens, T, pad):
     rng = np.random.default_rng(5)
     B = len(seq_lens)
