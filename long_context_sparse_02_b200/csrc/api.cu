@@ -103,6 +103,7 @@ bool attn_shape_ok(int Dqk, int Dv) { return (Dqk == 576 && Dv == 512) || (Dqk =
 size_t ld_of(int32_t max_len) { return align_up((size_t)max_len, 4); }
 
 struct LayerWs {
+    uint32_t *score_hist;  // decode: the indexer's per-query score histogram (kept zeroed between calls)
     float *scores;
     int32_t *idx;
     void *topk_ws;
@@ -116,6 +117,10 @@ LayerWs carve_layer(const dsa_layer_args *a, void *ws) {
     LayerWs w{};
     uint8_t *p = static_cast<uint8_t *>(ws);
     size_t off = 0;
+    if (a->mode == DSA_MODE_DECODE) {
+        w.score_hist = reinterpret_cast<uint32_t *>(p + off);
+        off += align_up((size_t)a->T * SCORE_HIST_BINS * 4, 256);
+    }
     w.scores = reinterpret_cast<float *>(p + off);
     off += align_up((size_t)a->T * ld_of(a->max_len) * 4, 256);
     if (!a->idx_out) {
@@ -259,7 +264,7 @@ dsa_status layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes, dsa
     const PagedDev pg = paged_dev(&a->pg);
     const int64_t ld = (int64_t)ld_of(a->max_len);
     IndexerArgs ia{a->q_idx, a->w, a->k_idx_cache, pg, decode ? nullptr : a->q_seq, decode ? nullptr : a->q_pos,
-                   a->T, a->HI, a->DI, a->max_len, lw.scores, ld};
+                   a->T, a->HI, a->DI, a->max_len, lw.scores, ld, decode ? lw.score_hist : nullptr};
     if (!mark(0)) return DSA_ERR_CUDA;
     dsa_status s = launch_indexer(ia, st);
     if (s != DSA_OK) return s;
@@ -268,13 +273,7 @@ dsa_status layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes, dsa
                 decode ? (int32_t)ROWLEN_SEQ_LENS : (int32_t)ROWLEN_QPOS_PLUS_1,
                 a->T, a->K, a->max_len, lw.idx, lw.topk_ws, lw.topk_bytes};
     ta.pdl = true;
-    if (decode) {  // the attention reads the kept rows next: start bringing them into L2
-        ta.pf_kv = static_cast<const uint8_t *>(static_cast<const void *>(a->kv_cache));
-        ta.pf_block_table = a->pg.block_table;
-        ta.pf_max_blocks = a->pg.max_blocks_per_seq;
-        ta.pf_num_pages = a->pg.num_pages;
-        ta.pf_row_bytes = a->Dqk * 2;
-    }
+    if (decode) ta.hist = lw.score_hist;
     s = launch_topk(ta, st);
     if (s != DSA_OK) return s;
     if (!mark(2)) return DSA_ERR_CUDA;

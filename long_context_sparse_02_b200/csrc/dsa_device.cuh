@@ -301,6 +301,9 @@ __device__ __forceinline__ uint4 dsmem_ld_v4(uint32_t remote) {
                  : "memory");
     return v;
 }
+__device__ __forceinline__ void dsmem_st(uint32_t remote, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
+}
 __device__ __forceinline__ void dsmem_red_add(uint32_t remote, uint32_t v) {
     asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
 }
@@ -322,9 +325,8 @@ __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.w
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-// Brings `bytes` (multiple of 16) at a 16-byte aligned global address into L2.
-__device__ __forceinline__ void l2_prefetch(const void *p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+__device__ __forceinline__ void red_add_global(uint32_t *p, uint32_t v) {
+    asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 // ---- misc -------------------------------------------------------------------------

@@ -45,7 +45,12 @@ struct IndexerArgs {
     int32_t T, HI, DI, max_len;
     float *scores;
     int64_t ld;
+    // optional (decode convention only): per-query histogram [T][SCORE_HIST_BINS]
+    // of score_key(score) >> SCORE_HIST_SHIFT, added to (it must hold zeros)
+    uint32_t *hist;
 };
+constexpr int SCORE_HIST_BINS = 2048;
+constexpr int SCORE_HIST_SHIFT = 21;
 dsa_status launch_indexer(const IndexerArgs &a, cudaStream_t st);
 
 // ---- top-K ---------------------------------------------------------------------
@@ -59,12 +64,10 @@ struct TopkArgs {
     int32_t *idx;
     void *ws;
     size_t ws_bytes;
-    // optional (decode rows, row r = sequence r): the latent cache rows of the
-    // kept positions are prefetched into L2 for the attention that follows
-    const uint8_t *pf_kv;  // NULL: no prefetch
-    const int32_t *pf_block_table;
-    int32_t pf_max_blocks, pf_num_pages, pf_row_bytes;
     bool pdl;  // launched as a programmatic dependent of the previous kernel
+    // optional: the indexer's per-row histogram of score_key >> SCORE_HIST_SHIFT
+    // ([R][SCORE_HIST_BINS]); read, then cleared to zeros for the next call
+    uint32_t *hist;
 };
 size_t topk_workspace_bytes(int32_t R, int32_t K, int32_t max_row_len);
 int topk_kernel_launches(int32_t R, int32_t max_row_len);

@@ -92,6 +92,7 @@ struct IdxParams {
     float *scores;
     int64_t ld;
     uint32_t *err;
+    uint32_t *hist;  // [T][SCORE_HIST_BINS] or NULL (decode kernel only)
 };
 
 // ============================================================================
@@ -103,7 +104,7 @@ struct IdxParams {
 template <int DI, int NH>
 struct DecCfg {
     static constexpr int CTAS_PER_SM = 2;
-    static constexpr int STAGES = DI == 128 ? 6 : 12;  // key tiles in flight per CTA
+    static constexpr int STAGES = DI == 128 ? 5 : 10;  // key tiles in flight per CTA
     static constexpr int EPI_GROUPS = 2;  // epilogue warpgroups, alternate tiles
     static constexpr int ACC = NH <= 32 ? 8 : 4;  // TMEM: ACC * NH <= 256 columns per CTA
     static constexpr int THREADS = 64 + 128 * EPI_GROUPS;
@@ -114,7 +115,11 @@ struct DecCfg {
     static constexpr uint32_t SBO = 8 * DI;
     static constexpr int MAXT = 1024;
     static constexpr int BAR_BYTES = 8 * (2 * STAGES + 2 * ACC + 4 + 1);
-    static constexpr int SMEM = 1024 + STAGES * A_BYTES + 2 * B_BYTES + BAR_BYTES + 4 * (MAXT + 1) + 16;
+    static constexpr int HIST_WORDS = SCORE_HIST_BINS / 2;  // per epilogue warpgroup: packed 16-bit counts
+    static constexpr int HIST_FLUSH_TILES = 256;            // a count stays below 2^16
+    static constexpr int SMEM =
+        1024 + STAGES * A_BYTES + 2 * B_BYTES + BAR_BYTES + 4 * (MAXT + 1) + 16 + 4 * EPI_GROUPS * HIST_WORDS;
+    static_assert(HIST_FLUSH_TILES * 128 < 65536, "packed counts do not carry");
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "tile alignment");
 };
 
@@ -147,9 +152,12 @@ __global__ void __launch_bounds__(DecCfg<DI, NH>::THREADS, DecCfg<DI, NH>::CTAS_
     int32_t *tstart = reinterpret_cast<int32_t *>(drain + 1);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tstart + C::MAXT + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    uint32_t *hist_sm = reinterpret_cast<uint32_t *>(tmem_slot + 4);  // [EPI_GROUPS][HIST_WORDS]
 
     const int warp = warp_id(), lane = lane_id();
     const int T = p.T;
+    if (p.hist)
+        for (int i = threadIdx.x; i < C::EPI_GROUPS * C::HIST_WORDS; i += blockDim.x) hist_sm[i] = 0;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
@@ -310,6 +318,8 @@ __global__ void __launch_bounds__(DecCfg<DI, NH>::THREADS, DecCfg<DI, NH>::CTAS_
         mbar_wait(drain, 0, p.err, nullptr);
     } else if (warp >= 2 && n > 0) {
         // ---------------- epilogue: warpgroup eg takes tiles i with i % EPI_GROUPS == eg ----------------
+        // Every thread of a warpgroup walks the same tiles (a failed wait only
+        // turns the work off), so the warpgroup's named barriers stay uniform.
         const int eg = (warp - 2) >> 2;
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
@@ -319,6 +329,25 @@ __global__ void __launch_bounds__(DecCfg<DI, NH>::THREADS, DecCfg<DI, NH>::CTAS_
         int tw = -1;  // query whose w is in registers
         QInfo qi{0, -1};
         float wr[NH];
+        bool alive = true;
+        // score histogram of this warpgroup's tiles of query hq (packed 16-bit counts)
+        uint32_t *hw = hist_sm + eg * C::HIST_WORDS;
+        int hq = -1, htiles = 0;
+        auto hflush = [&]() {
+            named_bar_sync(1 + eg, 128);  // every add of the warpgroup has landed
+            if (hq >= 0 && alive)
+                for (int wi = row; wi < C::HIST_WORDS; wi += 128) {
+                    const uint32_t v = hw[wi];
+                    if (v) {
+                        uint32_t *g = p.hist + (int64_t)hq * SCORE_HIST_BINS + 2 * wi;
+                        if (v & 0xFFFFu) red_add_global(g, v & 0xFFFFu);
+                        if (v >> 16) red_add_global(g + 1, v >> 16);
+                        hw[wi] = 0;
+                    }
+                }
+            htiles = 0;
+            named_bar_sync(1 + eg, 128);  // cleared before the next adds
+        };
         for (int i = 0; i < n; ++i) {
             if (i % C::EPI_GROUPS == eg) {
                 if (t != tw) {
@@ -327,9 +356,17 @@ __global__ void __launch_bounds__(DecCfg<DI, NH>::THREADS, DecCfg<DI, NH>::CTAS_
 #pragma unroll
                     for (int h = 0; h < NH; ++h) wr[h] = h < p.HI ? p.w[(int64_t)t * p.HI + h] : 0.f;
                 }
+                if (p.hist && (t != hq || htiles == C::HIST_FLUSH_TILES)) {
+                    hflush();
+                    hq = t;
+                }
+                ++htiles;
                 const int a = i % C::ACC;
                 const uint32_t aph = (i / C::ACC) & 1;
-                if (!mbar_wait(&tfull[a], aph, p.err, abort_flag)) break;
+                if (alive && !mbar_wait(&tfull[a], aph, p.err, abort_flag)) alive = false;
+            }
+            if (i % C::EPI_GROUPS == eg && alive) {
+                const int a = i % C::ACC;
                 tc_fence_after();
                 uint32_t r[NH];
                 const uint32_t ta = tmem + a * NH + lane_off;
@@ -348,13 +385,20 @@ __global__ void __launch_bounds__(DecCfg<DI, NH>::THREADS, DecCfg<DI, NH>::CTAS_
                 for (int h = 0; h < NH; ++h)
                     if (h < p.HI) sc = fmaf(wr[h], fmaxf(__uint_as_float(r[h]), 0.f), sc);
                 const int spos = j * 128 + row;
-                if (spos <= qi.last) p.scores[(int64_t)t * p.ld + spos] = sc;
+                if (spos <= qi.last) {
+                    p.scores[(int64_t)t * p.ld + spos] = sc;
+                    if (p.hist) {
+                        const uint32_t bin = score_key(sc) >> SCORE_HIST_SHIFT;
+                        atomicAdd(&hw[bin >> 1], 1u << ((bin & 1u) << 4));
+                    }
+                }
             }
             if (++j == tstart[t + 1] - tstart[t]) {
                 j = 0;
                 do { ++t; } while (t < T && tstart[t + 1] == tstart[t]);
             }
         }
+        if (p.hist) hflush();
     }
     tc_fence_before();
     __syncthreads();
@@ -698,7 +742,8 @@ dsa_status launch_indexer(const IndexerArgs &a, cudaStream_t st) {
     const DeviceInfo *dev = current_device();
     if (!dev) return DSA_ERR_CUDA;
     if (a.T == 0) return DSA_OK;
-    IdxParams p{a.w, a.q_seq, a.q_pos, a.pg, a.T, a.HI, a.max_len, a.scores, a.ld, dev->err};
+    IdxParams p{a.w, a.q_seq, a.q_pos, a.pg, a.T, a.HI, a.max_len, a.scores, a.ld, dev->err,
+                a.q_seq == nullptr ? a.hist : nullptr};
     const CUtensorMapSwizzle swz = a.DI == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUtensorMap km, qm;
     if (!make_tmap_2d(&km, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.DI, (uint64_t)a.pg.num_pages * 64, a.DI,

@@ -183,9 +183,9 @@ constexpr int RANK_MAX = 128;   // at most this many candidates: select by count
 // shared memory, in 32-bit words
 constexpr int CT_W_WORDS = CT_WARPS * 256;  // radix warp histograms | candidate lists
 constexpr int OWN_WORDS = LBINS / 2;        // bins owned by one CTA (CL >= 2)
-constexpr int PF_PAGES = 512;  // block-table entries staged for the L2 prefetch
+static_assert(2 * ((LBINS / 2 + 2 - 1) / 2) <= OWN_WORDS, "owned bins fit");
 constexpr int CT_FIXED_WORDS =
-    CT_W_WORDS + LBINS + OWN_WORDS + CT_WARPS * WCAP + 2 * 256 + 256 + CT_WARPS * 4 + 64 + PF_PAGES;
+    CT_W_WORDS + LBINS + OWN_WORDS + 2 * CT_WARPS * WCAP + 2 * 256 + 256 + CT_WARPS * 4 + 64;
 constexpr int CT_FIXED_SMEM = CT_FIXED_WORDS * 4;
 static_assert(CT_W_WORDS >= 2 * CAND_CAP, "candidate lists alias the radix histograms");
 static_assert(CT_FIXED_WORDS % 4 == 0, "the slice starts 16-byte aligned");
@@ -381,22 +381,33 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
     uint32_t *lhist = sm + CT_W_WORDS;     // [LBINS] this CTA's linear histogram
     uint32_t *own = lhist + LBINS;         // [LBINS / CL] cluster totals of the bins this CTA owns
     uint32_t *wlist = own + OWN_WORDS;     // [32][WCAP] per-warp listed positions
-    uint32_t *chist = wlist + CT_WARPS * WCAP;  // [2][256] radix path: this CTA's digit histogram
+    uint32_t *wkey = wlist + CT_WARPS * WCAP;  // [32][WCAP] their keys (histogram path)
+    uint32_t *chist = wkey + CT_WARPS * WCAP;  // [2][256] radix path: this CTA's digit histogram
     uint32_t *lcnt = chist;                // [32] binned path: listed positions per warp
     uint32_t *tot = chist + 2 * 256;       // [256] digit histogram
     uint32_t *wcnt = tot + 256;            // [32][4] per-warp scratch
     uint32_t *misc = wcnt + CT_WARPS * 4;  // [64] scalars (see above)
-    int32_t *pf_pages = reinterpret_cast<int32_t *>(misc + 64);  // [PF_PAGES] cache pages of the slice
-    float *xs = reinterpret_cast<float *>(pf_pages + PF_PAGES);  // [slice] the scores
-    constexpr int W = LBINS / CL;          // bins owned per CTA
+    float *xs = reinterpret_cast<float *>(misc + 64);  // [slice] the scores
+    constexpr int W = 2 * ((LBINS / 2 + CL - 1) / CL);  // bins owned per CTA (even: bin pairs share an owner)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t crank = CL > 1 ? cluster_ctarank() : 0;
     const int r = blockIdx.x / CL;
     const int n = row_length(a, r, crank == 0 ? err : nullptr);
     int32_t *out = a.idx + (int64_t)r * a.K;
+    // This CTA's share of the row's score histogram is cleared for the next
+    // call once every CTA of the cluster has read it.
+    auto clear_hist_share = [&]() {
+        uint32_t *hr = a.hist + (int64_t)r * SCORE_HIST_BINS;
+        for (int i = (int)crank * SCORE_HIST_BINS / CL + tid; i < ((int)crank + 1) * SCORE_HIST_BINS / CL; i += CT_THREADS)
+            hr[i] = 0;
+    };
     if (n <= a.K) {  // uniform across the cluster: every CTA returns here
         const int per = (a.K + CL - 1) / CL;
         for (int j = crank * per + tid; j < min(a.K, (int)(crank + 1) * per); j += CT_THREADS) out[j] = j < n ? j : -1;
+        if (a.hist) {
+            pdl_wait();  // the histogram is complete
+            clear_hist_share();
+        }
         return;
     }
     const int len = ((n + CL - 1) / CL + 3) & ~3;  // slices start 4 keys apart
@@ -404,23 +415,291 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
     const int m = min(n, s0 + len) - s0;
     const float *row = a.scores + (int64_t)r * a.ld + s0;
     pdl_trigger();
-    // block-table entries of the slice, for the L2 prefetch of kept rows
-    const int pf_page0 = s0 >> 6;
-    const bool pf = a.pf_kv != nullptr && m > 0 && ((s0 + m - 1) >> 6) - pf_page0 < PF_PAGES;
-    if (pf)
-        for (int i = tid; i <= ((s0 + m - 1) >> 6) - pf_page0; i += CT_THREADS) {
-            const int lp = pf_page0 + i;
-            const int pg = lp < a.pf_max_blocks ? a.pf_block_table[(int64_t)r * a.pf_max_blocks + lp] : -1;
-            pf_pages[i] = (pg >= 0 && pg < a.pf_num_pages) ? pg : -1;
-        }
     pdl_wait();  // the scores come from the previous kernel
 
+    bool fast_done = false, final_wait = CL > 1;
+    if (a.hist) {
+        // ---- histogram path.  The indexer counted the row's keys by their
+        // top bits (coarse bins).  Every CTA finds the coarse bin B of the
+        // K-th largest key from those counts; one pass over the slice lists,
+        // per warp and in position order, every position whose coarse bin is
+        // >= B with its key, and bins the keys of B into LBINS equal-width
+        // fine bins over B's score range; the fine counts meet in their owner
+        // CTAs (barrier 2); every CTA picks the fine bin of the K-th largest
+        // key; each CTA then stores its counts and its keys of that fine bin
+        // into every CTA of the cluster (barrier 3), after which all the rest
+        // is local: an exact select among those few keys and the compaction.
+        // Counts that do not add up to the row length (a workspace not
+        // cleared yet), a non-finite bin range or a full list take the full
+        // path below.
+        constexpr int CPR = CAND_CAP / 16;  // keys of the fine bin per CTA, stored at [rank][CPR]
+        const uint32_t *hr = a.hist + (int64_t)r * SCORE_HIST_BINS;
+        const int hb0 = SCORE_HIST_BINS - 1 - 2 * tid, hb1 = hb0 - 1;
+        const uint2 hv = *reinterpret_cast<const uint2 *>(hr + hb1);  // first: its latency hides behind the slice's
+        if (CL > 1) {
+            for (int i = tid; i < W; i += CT_THREADS) own[i] = 0;
+            cluster_arrive();  // own[] is clear before any CTA adds into it (paired wait below)
+        }
+        for (int i = tid; i < LBINS; i += CT_THREADS) lhist[i] = 0;
+        // the slice, 128 keys per warp step, loaded before anything waits on it
+        constexpr int NSTEP = 4;
+        const int per4 = ((m + CT_WARPS - 1) / CT_WARPS + 127) & ~127;
+        const int w0 = warp * per4, w1 = min(m, w0 + per4);
+        const bool vec = (reinterpret_cast<uintptr_t>(row) & 15u) == 0;
+        // uniform across the cluster: judged on the common slice length, not this CTA's m
+        const bool fits = (((len + CT_WARPS - 1) / CT_WARPS + 127) & ~127) <= NSTEP * 128;
+        float xv[NSTEP][4];
+        if (fits) {
+#pragma unroll
+            for (int st = 0; st < NSTEP; ++st) {
+                const int i0 = w0 + st * 128 + 4 * lane;
+                if (vec && i0 + 3 < w1) {
+                    const float4 v = *reinterpret_cast<const float4 *>(row + i0);
+                    xv[st][0] = v.x, xv[st][1] = v.y, xv[st][2] = v.z, xv[st][3] = v.w;
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) xv[st][k] = i0 + k < w1 ? row[i0 + k] : 0.f;
+                }
+            }
+        }
+        const uint32_t v0 = hv.y, v1 = hv.x, Ku = (uint32_t)a.K;
+        const bool sane = __syncthreads_and(v0 <= (uint32_t)n && v1 <= (uint32_t)n) != 0;
+        const uint32_t incl = ct_incl_scan(v0 + v1, wcnt);
+        const uint32_t total = wcnt[CT_WARPS - 1];
+        const uint32_t excl = incl - v0 - v1;
+        if (sane && total == (uint32_t)n && excl < Ku && Ku <= incl) {
+            const bool first = excl + v0 >= Ku;
+            misc[0] = first ? hb0 : hb1;
+            misc[1] = first ? excl : excl + v0;
+        }
+        if (tid == 0) misc[22] = 0;
+        __syncthreads();
+        const uint32_t B = misc[0], aboveB = misc[1];
+        const float xlo = key_score(B << SCORE_HIST_SHIFT), xhi = key_score(((B + 1) << SCORE_HIST_SHIFT) - 1u);
+        const float fscale = __fdiv_rn((float)LBINS, __fsub_rn(xhi, xlo));
+        // uniform across the cluster: the same counts and bin everywhere
+        const bool go = fits && sane && total == (uint32_t)n && isfinite(xlo) && isfinite(xhi) && xhi > xlo &&
+                        isfinite(fscale);
+        if (!go) {
+            if (CL > 1) cluster_wait();
+        } else {
+            uint32_t *wl = wlist + warp * WCAP, *wk = wkey + warp * WCAP;
+            uint32_t cnt = 0;
+            const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+            for (int st = 0; st < NSTEP; ++st) {
+                const int i0 = w0 + st * 128 + 4 * lane;
+                uint32_t key[4], selm = 0;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    key[k] = score_key(xv[st][k]);
+                    const uint32_t cb = key[k] >> SCORE_HIST_SHIFT;
+                    if (i0 + k < w1 && cb >= B) {
+                        selm |= 1u << k;
+                        if (cb == B) atomicAdd(&lhist[linear_bin(xv[st][k], xlo, fscale)], 1u);
+                    }
+                }
+                // list slot of this lane's first key: every selected key of the lower lanes comes first
+                uint32_t before = 0, stot = 0;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t bk = __ballot_sync(0xffffffffu, (selm >> k) & 1u);
+                    before += __popc(bk & lt);
+                    stot += __popc(bk);
+                }
+                uint32_t so = cnt + before;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if ((selm >> k) & 1u) {
+                        if (so < (uint32_t)WCAP) {
+                            wl[so] = (uint32_t)(i0 + k);
+                            wk[so] = key[k];
+                        }
+                        ++so;
+                    }
+                cnt += stot;
+            }
+            if (lane == 0) {
+                lcnt[warp] = cnt;
+                if (cnt > (uint32_t)WCAP) misc[22] = 1;
+            }
+            __syncthreads();  // the fine histogram of this CTA is complete
+            if (CL > 1) {
+                cluster_wait();  // every CTA's own[] is clear
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int bin = tid + h * CT_THREADS;
+                    const uint32_t v = lhist[bin];
+                    if (v) dsmem_red_add(dsmem_addr(own + bin % W, bin / W), v);
+                }
+            }
+            ct_cluster_or_block_sync<CL>();  // barrier 2: every fine total and overflow flag is in place
+            // the fine bin of the K-th largest key among bin B's keys (thread t: fine bins LBINS-1-2t, LBINS-2-2t)
+            const int fb0 = LBINS - 1 - 2 * tid, fb1 = fb0 - 1;
+            uint2 t2;
+            if (CL > 1) t2 = dsmem_ld_v2(dsmem_addr(own + fb1 % W, fb1 / W));
+            else t2 = make_uint2(lhist[fb1], lhist[fb0]);
+            const uint32_t f0 = t2.y, f1 = t2.x, rem = Ku - aboveB;
+            uint32_t ovf = 0;
+            if (warp == 0 && lane < CL) ovf = CL > 1 ? ld_dsmem_u32(misc + 22, lane) : misc[22];
+            const uint32_t fincl = ct_incl_scan(f0 + f1, wcnt);
+            const uint32_t fexcl = fincl - f0 - f1;
+            if (fexcl < rem && rem <= fincl) {
+                const bool first = fexcl + f0 >= rem;
+                misc[8] = first ? fb0 : fb1;
+                misc[9] = first ? fexcl : fexcl + f0;
+                misc[10] = first ? f0 : f1;
+            }
+            if (warp == 0) {
+                const bool any_ovf = __any_sync(0xffffffffu, ovf != 0);
+                if (lane == 0) misc[26] = any_ovf;
+            }
+            if (tid == 0) {
+                misc[2] = 0;   // candidates of this CTA
+                misc[20] = 0;  // keys of this CTA above the threshold fine bin
+            }
+            __syncthreads();
+            if (misc[26] == 0) {  // uniform across the cluster; else every CTA takes the full path
+                const int fb = (int)misc[8];
+                const uint32_t abovef = misc[9], Cf = misc[10];
+                // this CTA's candidates (fine bin fb of B), stored into every CTA at [crank][CPR]
+                const int wn = (int)lcnt[warp];
+                uint32_t nab = 0;
+                for (int j0 = 0; j0 < wn; j0 += 32) {
+                    const int j = j0 + lane;
+                    const uint32_t k = j < wn ? wk[j] : 0u;
+                    int f = -1;
+                    bool ab = false;
+                    if (j < wn) {
+                        if ((k >> SCORE_HIST_SHIFT) > B) ab = true;
+                        else {
+                            f = linear_bin(key_score(k), xlo, fscale);
+                            ab = f > fb;
+                        }
+                    }
+                    nab += __popc(__ballot_sync(0xffffffffu, ab));
+                    const bool isc = f == fb;
+                    const uint32_t cm = __ballot_sync(0xffffffffu, isc);
+                    if (cm) {
+                        uint32_t base = 0;
+                        if (lane == 0) base = atomicAdd(&misc[2], (uint32_t)__popc(cm));
+                        base = __shfl_sync(0xffffffffu, base, 0);
+                        const uint32_t slot = base + __popc(cm & lt);
+                        if (isc && slot < (uint32_t)CPR)
+                            for (int q = 0; q < CL; ++q) {
+                                uint32_t *dst = cand_all + crank * CPR + slot;
+                                if (CL > 1) dsmem_st(dsmem_addr(dst, q), k);
+                                else *dst = k;
+                            }
+                    }
+                }
+                if (lane == 0) atomicAdd(&misc[20], nab);
+                __syncthreads();  // this CTA's counts are final
+                if (tid < CL) {   // (keys above, candidates) of this CTA into slot crank of every CTA
+                    if (CL > 1) {
+                        dsmem_st(dsmem_addr(misc + 32 + crank, tid), misc[20]);
+                        dsmem_st(dsmem_addr(misc + 48 + crank, tid), misc[2]);
+                    } else {
+                        misc[32] = misc[20];
+                        misc[48] = misc[2];
+                    }
+                }
+                ct_cluster_or_block_sync<CL>();  // barrier 3: every count and key is stored everywhere
+                if (warp == 0) {
+                    // the candidates in rank order, contiguous; the counts of the earlier ranks
+                    uint32_t hq = lane < CL ? misc[32 + lane] : 0u, cq = lane < CL ? misc[48 + lane] : 0u;
+                    const bool ovc = __any_sync(0xffffffffu, cq > (uint32_t)CPR);
+                    uint32_t hx = hq, cx = cq;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const uint32_t y0 = __shfl_up_sync(0xffffffffu, hx, o), y1 = __shfl_up_sync(0xffffffffu, cx, o);
+                        if (lane >= o) hx += y0, cx += y1;
+                    }
+                    const uint32_t ctot = __shfl_sync(0xffffffffu, cx, 31), htot = __shfl_sync(0xffffffffu, hx, 31);
+                    const uint32_t cbefore = __shfl_sync(0xffffffffu, cx - cq, crank);
+                    const uint32_t hbefore = __shfl_sync(0xffffffffu, hx - hq, crank);
+                    if (lane == 0) {
+                        misc[24] = hbefore;
+                        misc[25] = cbefore;
+                        misc[27] = ctot;
+                        // more keys in a CTA's fine bin than its slots, or counts that disagree
+                        // with the histograms: the full path (identical copies: uniform)
+                        misc[28] = ovc || ctot != Cf || htot != aboveB + abovef;
+                    }
+                    if (!ovc) for (int q = 0; q < CL; ++q) {
+                        const uint32_t cn = min(__shfl_sync(0xffffffffu, cq, q), (uint32_t)CPR);
+                        const uint32_t o = __shfl_sync(0xffffffffu, cx - cq, q);
+                        for (uint32_t i = lane; i < cn; i += 32) cand_local[o + i] = cand_all[q * CPR + i];
+                    }
+                }
+                __syncthreads();
+              if (misc[28] == 0) {
+                final_wait = false;  // no CTA reads or writes another's shared memory from here on
+                clear_hist_share();
+                const uint32_t C = misc[27];
+                select_among(cand_local, (int)C, rem - abovef, tot, wcnt, misc + 4);
+                const uint32_t tau = misc[4], need = misc[5];
+                const uint32_t hi_before = misc[24], c_before = misc[25];
+                uint32_t g = 0, e = 0;
+                for (int j = tid; j < (int)c_before; j += CT_THREADS) {
+                    g += cand_local[j] > tau;
+                    e += cand_local[j] == tau;
+                }
+                ct_sum2(g, e, wcnt, misc + 12);
+                const uint32_t gt_before = hi_before + misc[12], eq_before = misc[13];
+                // compaction of the listed positions, in position order
+                g = 0, e = 0;
+                for (int j0 = 0; j0 < wn; j0 += 32) {
+                    const int j = j0 + lane;
+                    const uint32_t k = j < wn ? wk[j] : 0u;
+                    g += __popc(__ballot_sync(0xffffffffu, j < wn && k > tau));
+                    e += __popc(__ballot_sync(0xffffffffu, j < wn && k == tau));
+                }
+                if (lane == 0) {
+                    wcnt[warp * 4 + 0] = g;
+                    wcnt[warp * 4 + 1] = e;
+                }
+                __syncthreads();
+                if (warp == 0) {
+                    const uint32_t gv = wcnt[lane * 4 + 0], ev = wcnt[lane * 4 + 1];
+                    uint32_t gi = gv, ei = ev;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const uint32_t xg = __shfl_up_sync(0xffffffffu, gi, o), xe = __shfl_up_sync(0xffffffffu, ei, o);
+                        if (lane >= o) gi += xg, ei += xe;
+                    }
+                    wcnt[lane * 4 + 2] = gi - gv;
+                    wcnt[lane * 4 + 3] = ei - ev;
+                }
+                __syncthreads();
+                uint32_t gcur = gt_before + wcnt[warp * 4 + 2], ecur = eq_before + wcnt[warp * 4 + 3];
+                for (int j0 = 0; j0 < wn; j0 += 32) {
+                    const int j = j0 + lane;
+                    const uint32_t k = j < wn ? wk[j] : 0u;
+                    const bool gt = j < wn && k > tau, eq = j < wn && k == tau;
+                    const uint32_t gm = __ballot_sync(0xffffffffu, gt), em = __ballot_sync(0xffffffffu, eq);
+                    const uint32_t mg = gcur + __popc(gm & lt), me = ecur + __popc(em & lt);
+                    if (gt || (eq && me < need)) {
+                        const int pos = s0 + (int)wl[j];
+                        const uint32_t slot = mg + min(me, need);
+                        if (slot < Ku) out[slot] = pos;
+                        else record_error(err, DSA_DEVERR_SHAPE);
+                    }
+                    gcur += __popc(gm);
+                    ecur += __popc(em);
+                }
+                fast_done = true;
+              }
+            }
+        }
+    }
+
+    if (!fast_done) {
     // ---- 1. load the slice; its key range.  Histograms and counters are
     // cleared here: barrier 1 orders that before any CTA adds into them.
     for (int i = tid; i < LBINS; i += CT_THREADS) lhist[i] = 0;
     if (CL > 1)
         for (int i = tid; i < W; i += CT_THREADS) own[i] = 0;
-    if (tid == 0) misc[2] = 0;
     uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
     {
         int done = 0;
@@ -482,6 +761,8 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
         }
     }
     ct_cluster_or_block_sync<CL>();  // cluster barrier 1: every CTA's range is published
+    if (a.hist) clear_hist_share();  // every CTA has read the histogram
+    if (tid == 0) misc[2] = 0;  // candidate counter: the histogram path's remote reads of it end before barrier 1
     if (warp == 0) {
         uint32_t g0 = 0xFFFFFFFFu, g1 = 0u;
         if (lane < CL) {
@@ -505,10 +786,6 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
         if (CL > 1) cluster_arrive();  // the range reads above were the last remote reads
         for (int i = tid; i < m && s0 + i < a.K; i += CT_THREADS) {
             out[s0 + i] = s0 + i;
-            if (pf) {
-                const int pos = s0 + i, pg = pf_pages[(pos >> 6) - pf_page0];
-                if (pg >= 0) l2_prefetch(a.pf_kv + ((int64_t)pg * 64 + (pos & 63)) * a.pf_row_bytes, a.pf_row_bytes);
-            }
         }
         if (CL > 1) cluster_wait();
         return;
@@ -750,15 +1027,12 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
             const uint32_t slot = mg + min(me, need);
             if (slot < (uint32_t)a.K) out[slot] = s0 + i;
             else record_error(err, DSA_DEVERR_SHAPE);
-            if (pf) {
-                const int pos = s0 + i, pg = pf_pages[(pos >> 6) - pf_page0];
-                if (pg >= 0) l2_prefetch(a.pf_kv + ((int64_t)pg * 64 + (pos & 63)) * a.pf_row_bytes, a.pf_row_bytes);
-            }
         }
         gcur += __popc(gm);
         ecur += __popc(em);
     }
-    if (CL > 1) cluster_wait();  // no CTA leaves while another may still read its shared memory
+    }  // full path
+    if (final_wait) cluster_wait();  // no CTA leaves while another may still read its shared memory
 }
 
 // ---------------------------------------------------------------------------
@@ -927,21 +1201,22 @@ cudaLaunchConfig_t cluster_cfg(int R, int smem, cudaStream_t st, cudaLaunchAttri
     return cfg;
 }
 
-// How many 16-CTA clusters of this kernel the device runs at once (0 when it
-// cannot), cached per device and shared-memory size.
-int max_active_clusters16(const DeviceInfo *dev, int smem) {
+// How many clusters of CL CTAs of this kernel the device runs at once (0
+// when it cannot), cached per device, size and shared-memory size.
+template <int CL>
+int max_active_clusters(const DeviceInfo *dev, int smem) {
     static std::mutex mu;
     static std::vector<std::pair<std::pair<int, int>, int>> memo;
     std::lock_guard<std::mutex> lk(mu);
     for (auto &e : memo)
         if (e.first.first == dev->device && e.first.second == smem) return e.second;
     int num = 0;
-    auto fn = topk_cluster_kernel<16>;
+    auto fn = topk_cluster_kernel<CL>;
     if (ensure_smem(reinterpret_cast<const void *>(fn), smem) &&
-        cudaFuncSetAttribute(reinterpret_cast<const void *>(fn), cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-            cudaSuccess) {
+        (CL <= 8 || cudaFuncSetAttribute(reinterpret_cast<const void *>(fn),
+                                         cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess)) {
         cudaLaunchAttribute attr[1];
-        cudaLaunchConfig_t cfg = cluster_cfg<16>(1, smem, 0, attr);
+        cudaLaunchConfig_t cfg = cluster_cfg<CL>(1, smem, 0, attr);
         if (cudaOccupancyMaxActiveClusters(&num, fn, &cfg) != cudaSuccess) num = 0;
     }
     cudaGetLastError();
@@ -949,14 +1224,19 @@ int max_active_clusters16(const DeviceInfo *dev, int smem) {
     return num;
 }
 
-// Few rows: 16 CTAs per row when every row's cluster runs at once, else 8.
-// Many rows (prefill): one CTA per row.  A row whose slice does not fit in
-// shared memory is split over more CTAs (up to 8); longer rows go to the
-// multi-launch path.
+// Few rows: 16 or 10 CTAs per row when every row's cluster runs at once
+// (the graphics-processing-cluster layout decides how many large clusters
+// fit), else 8.  Many rows (prefill): one CTA per row.  A row whose slice
+// does not fit in shared memory is split over more CTAs (up to 8); longer
+// rows go to the multi-launch path.
 ClusterPlan cluster_plan(int R, int max_row_len, const DeviceInfo *dev) {
     if (R * 16 <= dev->sm_count) {
         const int smem = cluster_smem(max_row_len, 16);
-        if (smem <= dev->max_smem_optin && max_active_clusters16(dev, smem) >= R) return ClusterPlan{16, smem};
+        if (smem <= dev->max_smem_optin && max_active_clusters<16>(dev, smem) >= R) return ClusterPlan{16, smem};
+    }
+    if (R * 10 <= dev->sm_count) {
+        const int smem = cluster_smem(max_row_len, 10);
+        if (smem <= dev->max_smem_optin && max_active_clusters<10>(dev, smem) >= R) return ClusterPlan{10, smem};
     }
     for (int cl = (R >= dev->sm_count / 2) ? 1 : 8; cl <= 8; cl *= 2) {
         const int smem = cluster_smem(max_row_len, cl);
@@ -985,6 +1265,7 @@ dsa_status launch_cluster(const TopkArgs &a, const ClusterPlan &cp, cudaStream_t
         case 2: return launch_cluster_t<2>(a, cp.smem, st, err);
         case 4: return launch_cluster_t<4>(a, cp.smem, st, err);
         case 8: return launch_cluster_t<8>(a, cp.smem, st, err);
+        case 10: return launch_cluster_t<10>(a, cp.smem, st, err);
         default: return launch_cluster_t<16>(a, cp.smem, st, err);
     }
 }

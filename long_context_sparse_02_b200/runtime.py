@@ -47,7 +47,8 @@ class LayerOnDevice:
                                     self.k_cache, self.q, self.kv_cache, self.gate, self.pg, self.q_seq, self.q_pos,
                                     case.K, case.Dv, case.sm_scale, self.max_len, self.out, self.idx, self.lse)
         self.ws_bytes = _lib.layer_workspace_bytes(self.args)
-        self.ws = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=d)
+        # zero-filled once: decode calls find the score histogram cleared and keep it so
+        self.ws = torch.zeros(max(self.ws_bytes, 256), dtype=torch.uint8, device=d)
 
     def forward(self):
         _lib.layer_forward(self.args, self.ws)
@@ -61,4 +62,5 @@ class LayerOnDevice:
     def scores(self) -> torch.Tensor:
         """The fp32 scores the last forward left at the head of the workspace."""
         ld = (self.max_len + 3) // 4 * 4
-        return self.ws[: self.case.T * ld * 4].view(torch.float32).view(self.case.T, ld)
+        off = (self.case.T * 2048 * 4 + 255) // 256 * 256 if self.decode else 0  # the decode score histogram
+        return self.ws[off: off + self.case.T * ld * 4].view(torch.float32).view(self.case.T, ld)

@@ -267,3 +267,37 @@ def test_layer_forward_matches_oracle(L, orc, name, make, decode):
     assert np.array_equal(lay.idx.cpu().numpy(), idx)
     assert_attn_close(bf16_to_np(lay.out), out)
     no_device_error(L)
+
+
+def test_layer_decode_topk_fallbacks(L, orc):
+    """Decode through dsa_layer_forward where the top-K cannot use the
+    indexer's score histogram: (1) the workspace starts as garbage, so the
+    counts do not add up to the row length and the first call takes the full
+    path (clearing the histogram); the second call takes the histogram path;
+    (2) sequence 0's key rows are reordered so its scores rise with position,
+    which crowds every kept position into the last warps' lists (more than a
+    warp's list holds) and sends the top-K to the full path after its sweep."""
+    from long_context_sparse_02_b200.runtime import LayerOnDevice
+    c = synth.decode_case(7, [100000, 9000], K=2048, HI=32)
+    pg = orc.Paged(c.seq_lens, c.block_table, 64, c.num_pages)
+    q_seq = np.arange(c.T, dtype=np.int32)
+    q_pos = (c.seq_lens - 1).astype(np.int32)
+    sc = orc.indexer_scores(c.q_idx, c.w, c.k_cache, pg, q_seq, q_pos)
+    n0 = int(c.seq_lens[0])
+    order = np.argsort(sc[0, :n0], kind="stable")
+    pages = c.block_table[0, np.arange(n0) // 64]
+    slots = np.arange(n0) % 64
+    kc = c.k_cache.copy()
+    kc[pages, slots] = c.k_cache[pages[order], slots[order]]
+    c.k_cache = kc
+    _, idx, out = orc.layer_forward(c.q_idx, c.w, c.k_cache, c.q, c.kv_cache, c.gate, pg, q_seq, q_pos, c.K, c.Dv,
+                                    c.sm_scale)
+    assert np.array_equal(idx[0], np.arange(n0 - c.K, n0))  # the rise put every kept key at the end
+    lay = LayerOnDevice(c, decode=True)
+    lay.ws.fill_(0xA5)
+    for call in range(2):
+        lay.forward()
+        torch.cuda.synchronize()
+        assert np.array_equal(lay.idx.cpu().numpy(), idx), call
+        assert_attn_close(bf16_to_np(lay.out), out)
+    no_device_error(L)
