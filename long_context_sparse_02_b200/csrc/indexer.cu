@@ -419,13 +419,16 @@ struct PreCfg {
     static constexpr int A_BYTES = 128 * DI;
     static constexpr int B_BYTES = N * DI;
     static constexpr int ASTAGES = DI == 128 ? 6 : 10;
-    static constexpr int TMEM_COLS = 512;  // two 256-column accumulators, one per epilogue warpgroup
-    static constexpr int THREADS = 64 + 256;
+    static constexpr int TMEM_COLS = 512;  // two 256-column accumulators
+    static constexpr int EPI_WG = 4;       // epilogue warpgroups: two per accumulator, one per column half
+    static constexpr int THREADS = 64 + 128 * EPI_WG;
     static constexpr uint32_t SWZ = DI == 128 ? SWZ_128B : SWZ_64B;
     static constexpr uint32_t SBO = 8 * DI;
     static constexpr int BAR_BYTES = 8 * (2 * ASTAGES + 4 + 4 + 1);
     static constexpr int TBL = 3 * G;  // three per-role copies of the group table
+    // + 16: up to 8 bytes to align the weights, then the TMEM slot and abort flag
     static constexpr int SMEM = 1024 + 2 * B_BYTES + ASTAGES * A_BYTES + BAR_BYTES + 4 * N + 8 * TBL + 16;
+    static_assert(N % 4 == 0 && (4 * N) % 8 == 0, "weights are read as float4; the tables stay 8-byte aligned");
 };
 
 // One role's view of a query group: token u's (sequence, last position).
@@ -478,7 +481,8 @@ __global__ void __launch_bounds__(PreCfg<DI, HI>::THREADS, 1)
     uint64_t *tfull = bempty + 2;
     uint64_t *tempty = tfull + 2;
     uint64_t *drain = tempty + 2;
-    float *wbuf = reinterpret_cast<float *>(drain + 1);
+    float *wbuf = reinterpret_cast<float *>(  // [N], 16-byte aligned: read as float4
+        (reinterpret_cast<uintptr_t>(drain + 1) + 15) & ~uintptr_t(15));
     int2 *tbl_p = reinterpret_cast<int2 *>(wbuf + C::N);
     int2 *tbl_m = tbl_p + G;
     int2 *tbl_e = tbl_m + G;
@@ -498,7 +502,7 @@ __global__ void __launch_bounds__(PreCfg<DI, HI>::THREADS, 1)
             mbar_init(&bfull[i], 1);
             mbar_init(&bempty[i], 1);
             mbar_init(&tfull[i], 1);
-            mbar_init(&tempty[i], 4);
+            mbar_init(&tempty[i], 8);  // the four warps of each of the accumulator's two warpgroups
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -635,50 +639,73 @@ __global__ void __launch_bounds__(PreCfg<DI, HI>::THREADS, 1)
             mbar_wait(drain, 0, p.err, nullptr);
         }
     } else {
-        // ---------------- epilogue: two warpgroups (warps 2..5, 6..9) ----------------
-        // Tile tc lives in TMEM buffer tc % 2 and is reduced by warpgroup tc % 2.
-        const int et = threadIdx.x - 64;  // 0..255
+        // ---------------- epilogue: four warpgroups (warps 2..17) ----------------
+        // Tile tc lives in TMEM buffer a = tc % 2; warpgroups 2a and 2a+1 reduce
+        // its column halves (warp w reads TMEM lane quarter w % 4).
+        constexpr int NT = C::EPI_WG * 128;
+        const int et = threadIdx.x - 64;  // 0..NT-1
         const int eg = et >> 7;
+        const int ab = eg >> 1, ch = eg & 1;
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+        constexpr int HALF = C::N / 2;  // columns per warpgroup
         int tc = 0;
         bool ok = true;
         for (int r = 0; ok; ++r) {
             const int g = group_of(r, cta, grid, ngroups);
             if (g < 0) break;
-            named_bar_sync(1, 256);
-            load_group_tbl(tbl_e, g, G, p, true, et, 256);
-            for (int i = et; i < C::N; i += 256) {
+            named_bar_sync(1, NT);
+            load_group_tbl(tbl_e, g, G, p, true, et, NT);
+            // halved weights: w * max(x, 0) = (w / 2) * (x + |x|) exactly (x + |x| is 2x or 0), so the
+            // ReLU runs on the FMA pipe as an add with an absolute-value operand
+            for (int i = et; i < C::N; i += NT) {
                 const int t = g * G + i / HI;
-                wbuf[i] = t < p.T ? p.w[(int64_t)t * HI + (i % HI)] : 0.f;
+                wbuf[i] = t < p.T ? 0.5f * p.w[(int64_t)t * HI + (i % HI)] : 0.f;
             }
-            named_bar_sync(1, 256);
+            named_bar_sync(1, NT);
             for (int u = 0; ok && u < G;) {
                 int u1, b;
                 const int nt = next_run(tbl_e, G, u, &u1, &b);
                 for (int kt = 0; kt < nt; ++kt, ++tc) {
                     const int a = tc & 1;
-                    if (a != eg) continue;
+                    if (a != ab) continue;
                     if (!mbar_wait(&tfull[a], (tc >> 1) & 1, p.err, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const int spos = kt * 128 + row;
-                    const uint32_t ta = tmem + a * C::N + lane_off;
+                    const uint32_t ta = tmem + a * C::N + ch * HALF + lane_off;
+                    // 32 columns at a time, the next chunk's TMEM load in flight while
+                    // this one is reduced; independent partial sums keep the FMA chains
+                    // short (sums of exact products: the order does not matter)
+                    uint32_t rr[2][32];
+                    tmem_ld32(ta, rr[0]);
+                    tmem_wait_ld();
                     float acc = 0.f;
 #pragma unroll
-                    for (int cc = 0; cc < C::N / 32; ++cc) {
-                        uint32_t rr[32];
-                        tmem_ld32(ta + 32 * cc, rr);
-                        tmem_wait_ld();
+                    for (int cc = 0; cc < HALF / 32; ++cc) {
+                        if (cc + 1 < HALF / 32) tmem_ld32(ta + 32 * (cc + 1), rr[(cc + 1) & 1]);
+                        const uint32_t *x = rr[cc & 1];
+                        const int col0 = ch * HALF + 32 * cc;  // first column of the chunk
                         if constexpr (HI >= 32) {
-                            const int tok = (cc * 32) / HI;
-                            const int h0 = (cc * 32) % HI;
+                            float wv[32];
 #pragma unroll
-                            for (int h = 0; h < 32; ++h)
-                                acc = fmaf(wbuf[tok * HI + h0 + h], fmaxf(__uint_as_float(rr[h]), 0.f), acc);
+                            for (int i = 0; i < 8; ++i) {
+                                const float4 w4 = *reinterpret_cast<const float4 *>(wbuf + col0 + 4 * i);
+                                wv[4 * i] = w4.x, wv[4 * i + 1] = w4.y, wv[4 * i + 2] = w4.z, wv[4 * i + 3] = w4.w;
+                            }
+                            const int tok = col0 / HI;
+                            const int h0 = col0 % HI;
+                            float2 ps[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+                            for (int h = 0; h < 32; h += 2) {
+                                const float x0 = __uint_as_float(x[h]), x1 = __uint_as_float(x[h + 1]);
+                                ps[(h >> 1) & 3].x = fmaf(wv[h], x0 + fabsf(x0), ps[(h >> 1) & 3].x);
+                                ps[(h >> 1) & 3].y = fmaf(wv[h + 1], x1 + fabsf(x1), ps[(h >> 1) & 3].y);
+                            }
+                            acc += ((ps[0].x + ps[0].y) + (ps[1].x + ps[1].y)) + ((ps[2].x + ps[2].y) + (ps[3].x + ps[3].y));
                             if (h0 + 32 == HI) {
                                 const int2 info = tbl_e[tok];
                                 if (tok >= u && tok < u1 && spos <= info.y)
@@ -686,18 +713,28 @@ __global__ void __launch_bounds__(PreCfg<DI, HI>::THREADS, 1)
                                 acc = 0.f;
                             }
                         } else {
+                            constexpr int NA = HI >= 8 ? 2 : 1;  // partial sums per token
 #pragma unroll
                             for (int uu = 0; uu < 32 / HI; ++uu) {
-                                const int tok = (cc * 32) / HI + uu;
-                                float sc = 0.f;
+                                const int tok = col0 / HI + uu;
+                                float2 ps[NA];
 #pragma unroll
-                                for (int h = 0; h < HI; ++h)
-                                    sc = fmaf(wbuf[tok * HI + h], fmaxf(__uint_as_float(rr[uu * HI + h]), 0.f), sc);
+                                for (int i = 0; i < NA; ++i) ps[i] = make_float2(0.f, 0.f);
+#pragma unroll
+                                for (int h = 0; h < HI; h += 2) {
+                                    const float2 w2 = *reinterpret_cast<const float2 *>(wbuf + col0 + uu * HI + h);
+                                    const float x0 = __uint_as_float(x[uu * HI + h]), x1 = __uint_as_float(x[uu * HI + h + 1]);
+                                    ps[(h >> 1) % NA].x = fmaf(w2.x, x0 + fabsf(x0), ps[(h >> 1) % NA].x);
+                                    ps[(h >> 1) % NA].y = fmaf(w2.y, x1 + fabsf(x1), ps[(h >> 1) % NA].y);
+                                }
+                                float sc = ps[0].x + ps[0].y;
+                                if constexpr (NA == 2) sc += ps[1].x + ps[1].y;
                                 const int2 info = tbl_e[tok];
                                 if (tok >= u && tok < u1 && spos <= info.y)
                                     p.scores[(int64_t)(g * G + tok) * p.ld + spos] = sc;
                             }
                         }
+                        if (cc + 1 < HALF / 32) tmem_wait_ld();
                     }
                     tc_fence_before();
                     __syncwarp();
@@ -706,7 +743,7 @@ __global__ void __launch_bounds__(PreCfg<DI, HI>::THREADS, 1)
                 u = u1;
             }
             // the epilogue warpgroups leave the group loop together
-            ok = !named_bar_or(1, 256, !ok || *abort_flag);
+            ok = !named_bar_or(1, NT, !ok || *abort_flag);
         }
     }
     tc_fence_before();
