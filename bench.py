@@ -440,22 +440,26 @@ def prefill_indexer_leg(args, flush, T=32768, with_peak=True):
             "algorithmic_flops": flops}
 
 
-def cpu_baseline_leg(case):
-    """The oracle as it stands on this host: one whole decode step of the
-    workload (every sequence, full context, all heads)."""
+def cpu_baseline_leg(case, min_seconds=10.0, max_steps=8):
+    """The oracle as it stands on this host: whole decode steps of the workload
+    (every sequence, full context, all heads), repeated until about
+    min_seconds of CPU work have run (at most max_steps)."""
     import numpy as np
     from oracle import oracle
     pg = oracle.Paged(case.seq_lens, case.block_table, case.page_size, case.num_pages)
-    t0 = time.perf_counter()
-    _, idx, out = oracle.layer_forward(case.q_idx, case.w, case.k_cache, case.q, case.kv_cache, case.gate, pg,
-                                       np.arange(case.T, dtype=np.int32), case.seq_lens - 1, case.K, case.Dv,
-                                       case.sm_scale)
-    dt = time.perf_counter() - t0
+    steps, dt = 0, 0.0
+    while steps < max_steps and (steps == 0 or dt < min_seconds):
+        t0 = time.perf_counter()
+        _, idx, out = oracle.layer_forward(case.q_idx, case.w, case.k_cache, case.q, case.kv_cache, case.gate, pg,
+                                           np.arange(case.T, dtype=np.int32), case.seq_lens - 1, case.K, case.Dv,
+                                           case.sm_scale)
+        dt += time.perf_counter() - t0
+        steps += 1
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     cores = int(os.environ.get("OMP_NUM_THREADS", cores))
-    return ({"value": round(case.T / dt, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+    return ({"value": round(steps * case.T / dt, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
              "seconds": round(dt, 2),
-             "sample": f"one full decode step of {case.name} ({case.T} sequences x {case.max_len} tokens, "
+             "sample": f"{steps} full decode steps of {case.name} ({case.T} sequences x {case.max_len} tokens, "
                        f"all heads) through oracle.c (fp64, OpenMP)"}, idx, out)
 
 
