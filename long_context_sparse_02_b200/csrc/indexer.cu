@@ -227,6 +227,9 @@ __global__ void __launch_bounds__(DecCfg<DI, NH>::THREADS, DecCfg<DI, NH>::CTAS_
         };
         int tq, p0, p1;
         lookup(lane, tq, p0, p1);
+        // keys are read once: let them leave L2 first, so the scores written
+        // meanwhile are still there for the top-K that follows
+        const uint64_t kpol = l2_policy_evict_first();
         int issued = 0, qo = -1, tprev = -1;
         bool ok = true;
         for (int base = 0; ok && base < n; base += 32) {
@@ -257,8 +260,8 @@ __global__ void __launch_bounds__(DecCfg<DI, NH>::THREADS, DecCfg<DI, NH>::CTAS_
                         const uint32_t bytes = (pg0 >= 0 ? 64 * DI : 0) + (pg1 >= 0 ? 64 * DI : 0);
                         if (bytes) {
                             mbar_expect_tx(&full[s], bytes);
-                            if (pg0 >= 0) tma_load_2d(A, &kmap, &full[s], 0, pg0 * 64);
-                            if (pg1 >= 0) tma_load_2d(A + 64 * DI, &kmap, &full[s], 0, pg1 * 64);
+                            if (pg0 >= 0) tma_load_2d_hint(A, &kmap, &full[s], 0, pg0 * 64, kpol);
+                            if (pg1 >= 0) tma_load_2d_hint(A + 64 * DI, &kmap, &full[s], 0, pg1 * 64, kpol);
                         } else {
                             mbar_arrive(&full[s]);
                         }
