@@ -330,6 +330,14 @@ __device__ __forceinline__ void cluster_arrive() {
 }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
+// A global store under a predicate, as one predicated instruction (no branch):
+// the address is formed whether or not the store happens.
+__device__ __forceinline__ void st_global_if(float *addr, float v, bool pred) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %2, 0;\n\t@p st.global.f32 [%0], %1;\n\t}" ::"l"(addr),
+                 "f"(v), "r"((uint32_t)pred)
+                 : "memory");
+}
+
 // ---- programmatic dependent launch -----------------------------------------------
 // A kernel launched with programmatic stream serialization may start before
 // the previous kernel of its stream has finished.  pdl_wait blocks until that

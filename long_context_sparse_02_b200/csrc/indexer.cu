@@ -711,8 +711,8 @@ __global__ void __launch_bounds__(PreCfg<DI, HI>::THREADS, 1)
                             acc += ((ps[0].x + ps[0].y) + (ps[1].x + ps[1].y)) + ((ps[2].x + ps[2].y) + (ps[3].x + ps[3].y));
                             if (h0 + 32 == HI) {
                                 const int2 info = tbl_e[tok];
-                                if (tok >= u && tok < u1 && spos <= info.y)
-                                    p.scores[(int64_t)(g * G + tok) * p.ld + spos] = acc;
+                                st_global_if(p.scores + (int64_t)(g * G + tok) * p.ld + spos, acc,
+                                             tok >= u && tok < u1 && spos <= info.y);
                                 acc = 0.f;
                             }
                         } else {
@@ -733,8 +733,8 @@ __global__ void __launch_bounds__(PreCfg<DI, HI>::THREADS, 1)
                                 float sc = ps[0].x + ps[0].y;
                                 if constexpr (NA == 2) sc += ps[1].x + ps[1].y;
                                 const int2 info = tbl_e[tok];
-                                if (tok >= u && tok < u1 && spos <= info.y)
-                                    p.scores[(int64_t)(g * G + tok) * p.ld + spos] = sc;
+                                st_global_if(p.scores + (int64_t)(g * G + tok) * p.ld + spos, sc,
+                                             tok >= u && tok < u1 && spos <= info.y);
                             }
                         }
                         if (cc + 1 < HALF / 32) tmem_wait_ld();
