@@ -724,11 +724,15 @@ __global__ void __launch_bounds__(PreCfg<DI, HI>::THREADS, 1)
 #pragma unroll
                                 for (int i = 0; i < NA; ++i) ps[i] = make_float2(0.f, 0.f);
 #pragma unroll
-                                for (int h = 0; h < HI; h += 2) {
-                                    const float2 w2 = *reinterpret_cast<const float2 *>(wbuf + col0 + uu * HI + h);
+                                for (int h = 0; h < HI; h += 4) {
+                                    const float4 w4 = *reinterpret_cast<const float4 *>(wbuf + col0 + uu * HI + h);
                                     const float x0 = __uint_as_float(x[uu * HI + h]), x1 = __uint_as_float(x[uu * HI + h + 1]);
-                                    ps[(h >> 1) % NA].x = fmaf(w2.x, x0 + fabsf(x0), ps[(h >> 1) % NA].x);
-                                    ps[(h >> 1) % NA].y = fmaf(w2.y, x1 + fabsf(x1), ps[(h >> 1) % NA].y);
+                                    const float x2 = __uint_as_float(x[uu * HI + h + 2]), x3 = __uint_as_float(x[uu * HI + h + 3]);
+                                    float2 &q0 = ps[(h >> 1) % NA], &q1 = ps[((h >> 1) + 1) % NA];
+                                    q0.x = fmaf(w4.x, x0 + fabsf(x0), q0.x);
+                                    q0.y = fmaf(w4.y, x1 + fabsf(x1), q0.y);
+                                    q1.x = fmaf(w4.z, x2 + fabsf(x2), q1.x);
+                                    q1.y = fmaf(w4.w, x3 + fabsf(x3), q1.y);
                                 }
                                 float sc = ps[0].x + ps[0].y;
                                 if constexpr (NA == 2) sc += ps[1].x + ps[1].y;
