@@ -185,7 +185,7 @@ constexpr int CT_W_WORDS = CT_WARPS * 256;  // radix warp histograms | candidate
 constexpr int OWN_WORDS = LBINS / 2;        // bins owned by one CTA (CL >= 2)
 static_assert(2 * ((LBINS / 2 + 2 - 1) / 2) <= OWN_WORDS, "owned bins fit");
 constexpr int CT_FIXED_WORDS =
-    CT_W_WORDS + LBINS + OWN_WORDS + 2 * CT_WARPS * WCAP + 2 * 256 + 256 + CT_WARPS * 4 + 64;
+    CT_W_WORDS + LBINS + OWN_WORDS + 2 * CT_WARPS * WCAP + 2 * 256 + 256 + CT_WARPS * 4 + 64 + 4;
 constexpr int CT_FIXED_SMEM = CT_FIXED_WORDS * 4;
 static_assert(CT_W_WORDS >= 2 * CAND_CAP, "candidate lists alias the radix histograms");
 static_assert(CT_FIXED_WORDS % 4 == 0, "the slice starts 16-byte aligned");
@@ -387,7 +387,8 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
     uint32_t *tot = chist + 2 * 256;       // [256] digit histogram
     uint32_t *wcnt = tot + 256;            // [32][4] per-warp scratch
     uint32_t *misc = wcnt + CT_WARPS * 4;  // [64] scalars (see above)
-    float *xs = reinterpret_cast<float *>(misc + 64);  // [slice] the scores
+    uint64_t *sbar = reinterpret_cast<uint64_t *>(misc + 64);  // the slice's bulk copy
+    float *xs = reinterpret_cast<float *>(misc + 68);          // [slice] the scores
     constexpr int W = 2 * ((LBINS / 2 + CL - 1) / CL);  // bins owned per CTA (even: bin pairs share an owner)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t crank = CL > 1 ? cluster_ctarank() : 0;
@@ -414,8 +415,22 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
     const int s0 = min(n, (int)crank * len);
     const int m = min(n, s0 + len) - s0;
     const float *row = a.scores + (int64_t)r * a.ld + s0;
+    // Histogram path: the slice arrives in one bulk copy (the copy engine keeps
+    // more of it in flight than per-thread loads do).
+    const bool bulk = a.hist != nullptr && m > 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15u) == 0 &&
+                      (a.ld & 3) == 0;
+    if (bulk && tid == 0) {
+        mbar_init(sbar, 1);
+        fence_mbar_init();
+    }
+    if (bulk) __syncthreads();  // the barrier is initialised before anyone waits on it
     pdl_trigger();
     pdl_wait();  // the scores come from the previous kernel
+    if (bulk && tid == 0) {
+        const uint32_t bytes = (uint32_t)((m + 3) & ~3) * 4u;
+        mbar_expect_tx(sbar, bytes);
+        bulk_load(xs, row, bytes, sbar);
+    }
 
     bool fast_done = false, final_wait = CL > 1;
     if (a.hist) {
@@ -445,20 +460,23 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
         constexpr int NSTEP = 4;
         const int per4 = ((m + CT_WARPS - 1) / CT_WARPS + 127) & ~127;
         const int w0 = warp * per4, w1 = min(m, w0 + per4);
-        const bool vec = (reinterpret_cast<uintptr_t>(row) & 15u) == 0;
         // uniform across the cluster: judged on the common slice length, not this CTA's m
-        const bool fits = (((len + CT_WARPS - 1) / CT_WARPS + 127) & ~127) <= NSTEP * 128;
+        // (and on the alignment of the score rows, which is common to every slice)
+        const bool fits = (((len + CT_WARPS - 1) / CT_WARPS + 127) & ~127) <= NSTEP * 128 &&
+                          (reinterpret_cast<uintptr_t>(a.scores) & 15u) == 0 && (a.ld & 3) == 0;
         float xv[NSTEP][4];
+        // the copy is waited for on every path: nothing else may write xs while it is in flight
+        if (bulk) mbar_wait(sbar, 0, err, nullptr);
         if (fits) {
 #pragma unroll
             for (int st = 0; st < NSTEP; ++st) {
                 const int i0 = w0 + st * 128 + 4 * lane;
-                if (vec && i0 + 3 < w1) {
-                    const float4 v = *reinterpret_cast<const float4 *>(row + i0);
+                if (i0 + 3 < w1) {
+                    const float4 v = *reinterpret_cast<const float4 *>(xs + i0);
                     xv[st][0] = v.x, xv[st][1] = v.y, xv[st][2] = v.z, xv[st][3] = v.w;
                 } else {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) xv[st][k] = i0 + k < w1 ? row[i0 + k] : 0.f;
+                    for (int k = 0; k < 4; ++k) xv[st][k] = i0 + k < w1 ? xs[i0 + k] : -INFINITY;
                 }
             }
         }
@@ -486,34 +504,44 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
             uint32_t *wl = wlist + warp * WCAP, *wk = wkey + warp * WCAP;
             uint32_t cnt = 0;
             const uint32_t lt = (1u << lane) - 1u;
+            // A key is listed when its coarse bin is >= B, that is when its score is
+            // >= xlo (keys are monotone in the score, xlo is finite here, and entries
+            // past the slice hold -inf).  Listed keys are a few percent of the row, so
+            // each key costs one compare; the list bookkeeping runs only in the warps
+            // that found some, and usually with one ballot (at most one listed key
+            // per lane).
 #pragma unroll
             for (int st = 0; st < NSTEP; ++st) {
                 const int i0 = w0 + st * 128 + 4 * lane;
-                uint32_t key[4], selm = 0;
+                uint32_t selm = 0;
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    key[k] = score_key(xv[st][k]);
-                    const uint32_t cb = key[k] >> SCORE_HIST_SHIFT;
-                    if (i0 + k < w1 && cb >= B) {
-                        selm |= 1u << k;
-                        if (cb == B) atomicAdd(&lhist[linear_bin(xv[st][k], xlo, fscale)], 1u);
+                for (int k = 0; k < 4; ++k) selm |= (xv[st][k] >= xlo ? 1u : 0u) << k;
+                const uint32_t anyl = __ballot_sync(0xffffffffu, selm != 0);
+                if (anyl == 0) continue;
+                // list slot of this lane's first key: every listed key of the lower lanes comes first
+                uint32_t before, stot;
+                if (__any_sync(0xffffffffu, (selm & (selm - 1u)) != 0)) {
+                    before = 0, stot = 0;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t bk = __ballot_sync(0xffffffffu, (selm >> k) & 1u);
+                        before += __popc(bk & lt);
+                        stot += __popc(bk);
                     }
-                }
-                // list slot of this lane's first key: every selected key of the lower lanes comes first
-                uint32_t before = 0, stot = 0;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint32_t bk = __ballot_sync(0xffffffffu, (selm >> k) & 1u);
-                    before += __popc(bk & lt);
-                    stot += __popc(bk);
+                } else {
+                    before = __popc(anyl & lt);
+                    stot = __popc(anyl);
                 }
                 uint32_t so = cnt + before;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     if ((selm >> k) & 1u) {
+                        const float x = xv[st][k];
+                        const uint32_t key = score_key(x);
+                        if ((key >> SCORE_HIST_SHIFT) == B) atomicAdd(&lhist[linear_bin(x, xlo, fscale)], 1u);
                         if (so < (uint32_t)WCAP) {
                             wl[so] = (uint32_t)(i0 + k);
-                            wk[so] = key[k];
+                            wk[so] = key;
                         }
                         ++so;
                     }
