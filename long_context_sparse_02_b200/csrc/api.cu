@@ -82,6 +82,19 @@ bool make_tmap_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_3d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, const uint64_t dims[3], uint64_t stride1,
+                  uint64_t stride2, const uint32_t box[3], CUtensorMapSwizzle swz) {
+    CUtensorMap probe;
+    if (!make_tmap_2d(&probe, base, dt, dims[0], dims[1], stride1, box[0], box[1], swz)) return false;  // loads the encoder
+    if ((stride2 & 15u) || dims[2] == 0) return false;
+    cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+    cuuint64_t strides[2] = {stride1, stride2};
+    cuuint32_t b[3] = {box[0], box[1], box[2]};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return g_encode(m, dt, 3, const_cast<void *>(base), d, strides, b, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace dsa
 
 using namespace dsa;

@@ -302,7 +302,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             const bool resc = m_new > m + 8.f;
             float alpha = 1.f;
             if (resc) {
-                alpha = exp2f(m - m_new);
+                alpha = ex2_approx(m - m_new);
                 l *= alpha;
                 m = m_new;
             }
@@ -310,8 +310,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             float lsum = 0.f;
 #pragma unroll
             for (int i = 0; i < C::NC; i += 2) {
-                const float p0 = x[i] == -INFINITY ? 0.f : exp2f(x[i] - m);
-                const float p1 = x[i + 1] == -INFINITY ? 0.f : exp2f(x[i + 1] - m);
+                const float p0 = x[i] == -INFINITY ? 0.f : ex2_approx(x[i] - m);
+                const float p1 = x[i + 1] == -INFINITY ? 0.f : ex2_approx(x[i + 1] - m);
                 pk[i / 2] = pack_bf16(p0, p1);
                 const __nv_bfloat162 bv = *reinterpret_cast<__nv_bfloat162 *>(&pk[i / 2]);
                 lsum += __bfloat162float(bv.x) + __bfloat162float(bv.y);
@@ -444,12 +444,12 @@ struct DecAttnCfg {
     static constexpr int P_BYTES = 2 * 128 * 128;  // [128 heads x 128 rows] bf16, two atoms
     static constexpr int RING = Q_BYTES > P_BYTES ? Q_BYTES : P_BYTES;
     static constexpr int TMEM_COLS = DV <= 128 ? 128 : DV <= 256 ? 256 : 512;
-    static constexpr int NBAR = NKB + 2 * QS + 4;
-    static constexpr int OUT_ROW = DV * 2 + 16;   // staged output row (padded: conflict-free)
-    static constexpr int OUT_BYTES = 128 * OUT_ROW;
-    static constexpr bool OUT_IN_C = OUT_BYTES <= C_BYTES;
-    static_assert(OUT_IN_C || OUT_BYTES <= RING, "output staging fits");
+    static constexpr int NBAR = NKB + 2 * QS + 5;
+    // the output is staged in the rows region once PV has consumed it: one
+    // [128 heads x 64 dims] 128-byte-swizzled box per 64 value dims
+    static_assert(NVB * KB_BYTES <= C_BYTES, "output staging fits in the rows region");
     static constexpr int DPW = DV / 4;            // value dims per worker warp in the epilogue
+    static constexpr bool DV_HALF_SPLIT = DV == 512;  // the epilogue halves: warps 0-7 dims < 256, 8-15 the rest
     static constexpr int SMEM = 1024 + C_BYTES + RING + 8 * NBAR + 8 * DEC_NR + 2 * 4 * 128 * 4 + 64;
     static_assert(DV >= 64 && DV % 64 == 0 && DV <= 512, "value width");
 };
@@ -473,7 +473,8 @@ struct DecAttnParams {
 // MMAs and owns TMEM; warp 17 streams Q.
 template <int DQK, int DV>
 __global__ void __launch_bounds__(DEC_THREADS, 1)
-    attn_decode_kernel(const __grid_constant__ CUtensorMap qmap, const DecAttnParams p) {
+    attn_decode_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap omap,
+                       const DecAttnParams p) {
     using C = DecAttnCfg<DQK, DV>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
@@ -484,8 +485,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
     uint64_t *q_empty = q_full + C::QS;                                 // [QS]
     uint64_t *s_full = q_empty + C::QS;
     uint64_t *p_full = s_full + 1;
-    uint64_t *o_full = p_full + 1;
-    uint64_t *drain = o_full + 1;
+    uint64_t *o_full = p_full + 1;  // [2]: O columns [0, 256) and [256, DV)
+    uint64_t *drain = o_full + 2;
     int64_t *rowid = reinterpret_cast<int64_t *>(drain + 1);  // [128] cache row of each selected entry, -1 = none
     float *red_m = reinterpret_cast<float *>(rowid + DEC_NR);  // [4][128] partial row maxima
     float *red_l = red_m + 4 * 128;                            // [4][128] partial sums
@@ -514,14 +515,16 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
             mbar_init(&q_empty[i], 1);
         }
         mbar_init(s_full, 1);
-        mbar_init(p_full, DEC_WORKERS);
-        mbar_init(o_full, 1);
+        mbar_init(p_full, 1);
+        mbar_init(&o_full[0], 1);
+        mbar_init(&o_full[1], 1);
         mbar_init(drain, 1);
         *any_valid = 0;
         *abort_flag = 0;
         if (!tok_ok) record_error(p.err, DSA_DEVERR_POSITION);
         fence_mbar_init();
         tma_prefetch_desc(&qmap);
+        tma_prefetch_desc(&omap);
     }
     if (warp == DEC_MMA_WARP) tmem_alloc(tmem_slot, C::TMEM_COLS);
     __syncthreads();
@@ -580,6 +583,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
         // ---------------- softmax: warp w = (head quarter w%4, row block w/4) ----------------
         const int qr = warp & 3, cb = warp >> 2;
         const int head = 32 * qr + lane;
+        // value dims of this warp's epilogue: [DV/4 * cb, DV/4 * (cb + 1)), in O half ohalf;
+        // warps 0-7 / 8-15 (threads 0-255 / 256-511) are the two halves when DV > 256
+        const int ohalf = C::DPW * cb >= 256 ? 1 : 0;
+        static_assert(C::DV_HALF_SPLIT || DV <= 256, "halves");
         const uint32_t lane_off = static_cast<uint32_t>(32 * qr) << 16;
         float m = -INFINITY;
         bool have_o = false;
@@ -607,8 +614,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
             float ls = 0.f;
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-                const float p0 = ((vm >> i) & 1u) ? exp2f(__uint_as_float(sr[i]) * p.scale_log2 - m) : 0.f;
-                const float p1 = ((vm >> (i + 1)) & 1u) ? exp2f(__uint_as_float(sr[i + 1]) * p.scale_log2 - m) : 0.f;
+                const float p0 = ((vm >> i) & 1u) ? ex2_approx(__uint_as_float(sr[i]) * p.scale_log2 - m) : 0.f;
+                const float p1 = ((vm >> (i + 1)) & 1u) ? ex2_approx(__uint_as_float(sr[i + 1]) * p.scale_log2 - m) : 0.f;
                 pk[i / 2] = pack_bf16(p0, p1);
                 const __nv_bfloat162 bv = *reinterpret_cast<__nv_bfloat162 *>(&pk[i / 2]);
                 ls += __bfloat162float(bv.x) + __bfloat162float(bv.y);
@@ -624,49 +631,61 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
-            have_o = mbar_wait(o_full, 0, p.err, abort_flag);
+            named_bar_sync(1, DEC_WORKER_THREADS);  // P and every partial sum are written
+            if (threadIdx.x == 0) mbar_arrive(p_full);
+            have_o = mbar_wait(&o_full[ohalf], 0, p.err, abort_flag);
             tc_fence_after();
         }
         // ---------------- epilogue: warp w = (head quarter w%4, value dims DV/4 * (w/4)..) ----------------
-        // every partial sum written; S, P and the rows are consumed; O is read by all or by none
-        have_o = !named_bar_or(1, DEC_WORKER_THREADS, go && !have_o) && go;
+        // every partial sum written; S, P and the rows are consumed; O is read by all or by none.
+        // O/l goes to the rows region as bf16 in the 128-byte-swizzled layout of
+        // the output map's [64 dims x 128 heads] boxes, then one tensor store per box.
+        // (per O half: the half's 256 worker threads agree; the halves do not wait for each other)
+        const uint32_t hbar = C::DV_HALF_SPLIT ? 2 + ohalf : 1;
+        const uint32_t hthreads = C::DV_HALF_SPLIT ? DEC_WORKER_THREADS / 2 : DEC_WORKER_THREADS;
+        have_o = !named_bar_or(hbar, hthreads, go && !have_o) && go;
         const float l = have_o ? red_l[head] + red_l[128 + head] + red_l[256 + head] + red_l[384 + head] : 0.f;
         const float inv = l > 0.f ? 1.f / l : 0.f;
         const int d0 = cb * C::DPW;
-        uint8_t *stg = (C::OUT_IN_C ? Cs : ring) + head * C::OUT_ROW + d0 * 2;
+        constexpr int STEP = C::DPW % 32 == 0 ? 32 : 16;  // TMEM columns read per wait
 #pragma unroll 1
-        for (int c0 = 0; c0 < C::DPW; c0 += 16) {
-            uint32_t o[16];
+        for (int c0 = 0; c0 < C::DPW; c0 += STEP) {
+            uint32_t o[STEP];
             if (have_o) {
-                tmem_ld16(tmem + d0 + c0 + lane_off, o);
+#pragma unroll
+                for (int h = 0; h < STEP; h += 16) tmem_ld16(tmem + d0 + c0 + h + lane_off, o + h);
                 tmem_wait_ld();
             } else {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) o[i] = 0u;
+                for (int i = 0; i < STEP; ++i) o[i] = 0u;
             }
 #pragma unroll
-            for (int i = 0; i < 16; i += 8) {
+            for (int i = 0; i < STEP; i += 8) {
+                const int d = d0 + c0 + i;
                 uint4 v;
                 v.x = pack_bf16(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
                 v.y = pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
                 v.z = pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
                 v.w = pack_bf16(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-                *reinterpret_cast<uint4 *>(stg + (c0 + i) * 2) = v;
+                *reinterpret_cast<uint4 *>(Cs + (d >> 6) * C::KB_BYTES + head * 128 +
+                                           ((((d & 63) >> 3) ^ (head & 7)) << 4)) = v;
             }
         }
         fence_proxy_async_smem();
-        named_bar_sync(1, DEC_WORKER_THREADS);  // the whole staged row is written
-        const bool live = head < p.H;
-        const int64_t prow = ((int64_t)t * p.splits + split) * p.H + head;
-        if (cb == 0 && live) {
-            bulk_store(p.part_o + prow * p.Dv, (C::OUT_IN_C ? Cs : ring) + head * C::OUT_ROW, DV * 2);
+        named_bar_sync(hbar, hthreads);  // every box of this half is staged
+        const bool issuer = threadIdx.x == (C::DV_HALF_SPLIT ? ohalf * (DEC_WORKER_THREADS / 2) : 0);
+        if (issuer) {  // heads >= H lie outside the map and are not written
+            const int b0 = C::DV_HALF_SPLIT ? ohalf * (C::NVB / 2) : 0;
+            const int b1 = C::DV_HALF_SPLIT ? b0 + C::NVB / 2 : C::NVB;
+            for (int bx = b0; bx < b1; ++bx) tma_store_3d(&omap, Cs + bx * C::KB_BYTES, bx * 64, 0, t * p.splits + split);
             bulk_commit();
+        }
+        if (cb == 0 && head < p.H) {
+            const int64_t prow = ((int64_t)t * p.splits + split) * p.H + head;
             p.part_ml[prow * 2 + 0] = m;
             p.part_ml[prow * 2 + 1] = l;
-            bulk_wait_read_all();
         }
+        if (issuer) bulk_wait_read_all();  // the staged boxes stay until the stores have read them
     } else if (warp == DEC_Q_WARP) {
         // ---------------- rest of the Q stream (TMA, from L2) ----------------
         if (lane == 0) {
@@ -712,8 +731,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
                     for (int k = 0; k < DEC_NR / 16; ++k)
                         mma_bf16(tmem + nb * 64, sdesc(r0 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, SWZ_128B),
                                  sdesc(c0 + nb * C::KB_BYTES + k * 2048, C::KB_BYTES, 1024, SWZ_128B), id_pv, k != 0);
+                    mma_commit(&o_full[nb / 4]);  // this half of O is complete
                 }
-                mma_commit(o_full);
+                if (C::NVB <= 4) mma_commit(&o_full[1]);
             }
             mma_commit(drain);
             mbar_wait(drain, 0, p.err, nullptr);
@@ -764,14 +784,14 @@ __global__ void __launch_bounds__(CMB_THREADS) attn_decode_combine_kernel(const 
         for (int u = 0; u < CMB_BATCH; ++u)
             if (v[u].y > 0.f) Mb = fmaxf(Mb, v[u].x);
         if (Mb == -INFINITY) continue;  // nothing selected so far
-        const float r = M == -INFINITY ? 0.f : exp2f(M - Mb);
+        const float r = M == -INFINITY ? 0.f : ex2_approx(M - Mb);
         W *= r;
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] *= r;
         M = Mb;
 #pragma unroll
         for (int u = 0; u < CMB_BATCH; ++u) {
-            const float w = v[u].y > 0.f ? v[u].y * exp2f(v[u].x - M) : 0.f;
+            const float w = v[u].y > 0.f ? v[u].y * ex2_approx(v[u].x - M) : 0.f;
             W += w;
             const uint32_t w4[4] = {o[u].x, o[u].y, o[u].z, o[u].w};
 #pragma unroll
@@ -808,7 +828,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
     float wsum = 0.f;
     for (int s = 0; s < S; ++s) {
         const float *ml = p.part_ml + (((int64_t)t * S + s) * p.H + h) * 2;
-        if (ml[1] > 0.f) wsum += ml[1] * exp2f(ml[0] - M);
+        if (ml[1] > 0.f) wsum += ml[1] * ex2_approx(ml[0] - M);
     }
     const float g = __bfloat162float(__ushort_as_bfloat16(p.gate[(int64_t)t * p.H + h]));
     const float sig = 1.f / (1.f + __expf(-g));
@@ -820,7 +840,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnParams p) {
             const int64_t prow = ((int64_t)t * S + s) * p.H + h;
             const float *ml = p.part_ml + prow * 2;
             if (!(ml[1] > 0.f)) continue;
-            const float c = ml[1] * exp2f(ml[0] - M);
+            const float c = ml[1] * ex2_approx(ml[0] - M);
             const float4 v = *reinterpret_cast<const float4 *>(p.part_o + prow * p.Dv + d0);
             acc.x = fmaf(c, v.x, acc.x);
             acc.y = fmaf(c, v.y, acc.y);
@@ -922,7 +942,14 @@ dsa_status run_attn_decode(const CUtensorMap &qm, const DecAttnParams &p, const 
     using C = DecAttnCfg<DQK, DV>;
     auto fn = attn_decode_kernel<DQK, DV>;
     if (!ensure_smem(reinterpret_cast<const void *>(fn), C::SMEM)) return DSA_ERR_CUDA;
-    if (launch_k(fn, dim3(p.splits, p.T), dim3(DEC_THREADS), C::SMEM, st, pdl, qm, p) != cudaSuccess)
+    // partials [T * splits][H][Dv] bf16, stored one [64 dims x H heads] box at a time
+    CUtensorMap om;
+    const uint64_t odims[3] = {(uint64_t)p.Dv, (uint64_t)p.H, (uint64_t)p.T * p.splits};
+    const uint32_t obox[3] = {64, (uint32_t)p.H, 1};
+    if (p.H > 128 || !make_tmap_3d(&om, p.part_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, odims, (uint64_t)p.Dv * 2,
+                                   (uint64_t)p.H * p.Dv * 2, obox, CU_TENSOR_MAP_SWIZZLE_128B))
+        return DSA_ERR_INVALID_ARG;
+    if (launch_k(fn, dim3(p.splits, p.T), dim3(DEC_THREADS), C::SMEM, st, pdl, qm, om, p) != cudaSuccess)
         return DSA_ERR_CUDA;
     const int64_t threads = (int64_t)p.T * p.H * (p.Dv / 8);
     return launch_k(attn_decode_combine_kernel, dim3((unsigned)((threads + CMB_THREADS - 1) / CMB_THREADS)),

@@ -157,6 +157,16 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
         : "memory");
 }
 
+// Shared -> global tensor store of one box (bulk async group); the smem image
+// must be made visible to the async proxy first.  Elements outside the
+// tensor are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int32_t x, int32_t y,
+                                             int32_t z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
+                 "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
 // Contiguous shared -> global copy (bulk async group); both addresses 16-byte
 // aligned, bytes % 16 == 0.  The smem must be made visible to the async proxy
 // first (fence_proxy_async_smem after the generic writes).
@@ -353,6 +363,15 @@ __device__ __forceinline__ void red_add_global(uint32_t *p, uint32_t v) {
 }
 
 // ---- misc -------------------------------------------------------------------------
+
+// 2^x by the hardware's approximate base-2 exponential (ex2.approx: relative
+// error about 2^-22, denormal results flushed to zero).  Softmax weights are
+// rounded to bf16 or merged into fp32 sums afterwards, so this is ample.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 __device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }

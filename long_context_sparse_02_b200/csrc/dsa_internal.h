@@ -25,6 +25,12 @@ const DeviceInfo *current_device();
 bool make_tmap_2d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
 
+// Builds a 3-D tiled tensor map: dims[0] elements of `elem_bytes` innermost,
+// then dims[1] rows `stride1` bytes apart, then dims[2] planes `stride2` bytes
+// apart; box [box0, box1, box2].
+bool make_tmap_3d(CUtensorMap *m, const void *base, CUtensorMapDataType dt, const uint64_t dims[3], uint64_t stride1,
+                  uint64_t stride2, const uint32_t box[3], CUtensorMapSwizzle swz);
+
 // Raises the dynamic shared-memory limit of `fn` once per device.
 bool ensure_smem(const void *fn, int bytes);
 
