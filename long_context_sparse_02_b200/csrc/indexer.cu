@@ -423,7 +423,7 @@ struct PreCfg {
     static constexpr int B_BYTES = N * DI;
     static constexpr int ASTAGES = DI == 128 ? 6 : 10;
     static constexpr int TMEM_COLS = 512;  // two 256-column accumulators
-    static constexpr int EPI_WG = 4;       // epilogue warpgroups: two per accumulator, one per column half
+    static constexpr int EPI_WG = 4;       // epilogue warpgroups: each reduces one column quarter of every tile
     static constexpr int THREADS = 64 + 128 * EPI_WG;
     static constexpr uint32_t SWZ = DI == 128 ? SWZ_128B : SWZ_64B;
     static constexpr uint32_t SBO = 8 * DI;
@@ -505,7 +505,7 @@ __global__ void __launch_bounds__(PreCfg<DI, HI>::THREADS, 1)
             mbar_init(&bfull[i], 1);
             mbar_init(&bempty[i], 1);
             mbar_init(&tfull[i], 1);
-            mbar_init(&tempty[i], 8);  // the four warps of each of the accumulator's two warpgroups
+            mbar_init(&tempty[i], 4 * C::EPI_WG);  // every epilogue warp
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -643,16 +643,18 @@ __global__ void __launch_bounds__(PreCfg<DI, HI>::THREADS, 1)
         }
     } else {
         // ---------------- epilogue: four warpgroups (warps 2..17) ----------------
-        // Tile tc lives in TMEM buffer a = tc % 2; warpgroups 2a and 2a+1 reduce
-        // its column halves (warp w reads TMEM lane quarter w % 4).
+        // Tile tc lives in TMEM buffer a = tc % 2; warpgroup eg reduces column
+        // quarter eg of every tile (warp w reads TMEM lane quarter w % 4), so
+        // while the MMA refills one buffer every epilogue warp works on the
+        // other one.
         constexpr int NT = C::EPI_WG * 128;
         const int et = threadIdx.x - 64;  // 0..NT-1
         const int eg = et >> 7;
-        const int ab = eg >> 1, ch = eg & 1;
         const int q4 = warp & 3;
         const int row = q4 * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-        constexpr int HALF = C::N / 2;  // columns per warpgroup
+        constexpr int HALF = C::N / C::EPI_WG;  // columns per warpgroup
+        const int ch = eg;
         int tc = 0;
         bool ok = true;
         for (int r = 0; ok; ++r) {
@@ -672,7 +674,6 @@ __global__ void __launch_bounds__(PreCfg<DI, HI>::THREADS, 1)
                 const int nt = next_run(tbl_e, G, u, &u1, &b);
                 for (int kt = 0; kt < nt; ++kt, ++tc) {
                     const int a = tc & 1;
-                    if (a != ab) continue;
                     if (!mbar_wait(&tfull[a], (tc >> 1) & 1, p.err, abort_flag)) {
                         ok = false;
                         break;
