@@ -62,7 +62,7 @@ PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "indexer_decode_B8_L131072.md")
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--seed", type=int, default=0)
@@ -143,6 +143,10 @@ class ClockSampler:
             time.sleep(self.period)
 
     def __enter__(self):
+        # the timed loop is a tight Python loop: let the sampler thread get the
+        # interpreter often enough to sample during it
+        self._switch = sys.getswitchinterval()
+        sys.setswitchinterval(0.0002)
         if self.ok:
             self._stop = threading.Event()
             self._t = threading.Thread(target=self._run, daemon=True)
@@ -153,6 +157,7 @@ class ClockSampler:
         if self.ok:
             self._stop.set()
             self._t.join()
+        sys.setswitchinterval(self._switch)
         return False
 
     def summary(self):
