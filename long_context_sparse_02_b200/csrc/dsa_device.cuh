@@ -181,6 +181,9 @@ __device__ __forceinline__ void bulk_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// Brings the line holding *p into L2 (no data returned, no fault on a valid address).
+__device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 // ---- 16-byte async copies (gathers) ---------------------------------------------
 
 __device__ __forceinline__ void cp_async_16(void *dst, const void *src) {

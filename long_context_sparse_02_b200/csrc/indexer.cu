@@ -156,6 +156,22 @@ __global__ void __launch_bounds__(DecCfg<DI, NH>::THREADS, DecCfg<DI, NH>::CTAS_
 
     const int warp = warp_id(), lane = lane_id();
     const int T = p.T;
+    if (threadIdx.x == 64 && p.q_seq == nullptr) {
+        // Warm L2 with what the producer's first lookups read (inputs of the
+        // layer, cold at launch): the sequence lengths, and the block-table
+        // lines of this CTA's share of the tiles as if every query had max_len
+        // keys (exact when the lengths are equal; a prefetch that misses costs nothing).
+        for (int i = 0; i < T; i += 32) prefetch_l2(p.pg.seq_lens + i);
+        const int64_t tq = (p.max_len + 127) >> 7;  // tiles per query at max_len
+        const int64_t tb = (int64_t)T * tq;
+        const int64_t k0 = tb * blockIdx.x / gridDim.x, k1 = tb * (blockIdx.x + 1) / gridDim.x;
+        for (int64_t k = k0; k < k1 + 16; k += 16) {  // 16 tiles = 32 pages = one 128-byte line of the table
+            const int64_t kk = k < k1 ? k : k1 - 1;
+            const int64_t q = kk / tq, j = kk % tq;
+            if (kk < k0 || q >= p.pg.num_seqs || 2 * j >= p.pg.max_blocks) break;
+            prefetch_l2(p.pg.block_table + q * p.pg.max_blocks + 2 * j);
+        }
+    }
     if (p.hist)
         for (int i = threadIdx.x; i < C::EPI_GROUPS * C::HIST_WORDS; i += blockDim.x) hist_sm[i] = 0;
 
