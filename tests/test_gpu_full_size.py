@@ -1,0 +1,117 @@
+"""CUDA path vs the CPU oracle at the workloads' full sizes, through the C ABI.
+
+The same calls and launch configurations the benchmark times:
+
+* decode, 8 sequences x 131072 tokens (32x128 indexer, K = 2048, 128 heads over
+  the 576-wide latent) through dsa_layer_forward -- every index and every
+  output element compared;
+* decode, one sequence of 1,048,576 tokens (the longest context; its top-K row
+  does not fit a cluster's shared memory) -- every index and output compared;
+* prefill indexer, one sequence of T = 32768 causal queries (16x128) through
+  dsa_indexer_scores and dsa_topk over all 32768 rows -- scores and indices of
+  sampled rows (the first, last and tile-boundary rows plus seeded random ones)
+  compared bit for bit with the oracle, which computes those rows alone;
+* the hybrid serving step: 64 decode sequences with lengths uniform in
+  [4096, 65536] through one DSA layer (16x128 indexer) and one sliding-window
+  layer (64 heads x 128, window 128) -- every element compared.
+
+Indexer inputs are dyadic, so scores and indices must match bit for bit;
+attention outputs within rtol 2e-2 / atol 1e-2 and a relative Frobenius error
+of at most 1e-2 (bf16 outputs).
+"""
+import numpy as np
+import pytest
+import torch
+
+from long_context_sparse_02_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+RTOL, ATOL, FRO = 2e-2, 1e-2, 1e-2
+
+
+@pytest.fixture(scope="module")
+def L():
+    from long_context_sparse_02_b200 import build
+    build.build()
+    from long_context_sparse_02_b200 import _lib
+    _lib.device_error(reset=True)
+    return _lib
+
+
+def dev(a):
+    from long_context_sparse_02_b200.runtime import to_dev
+    return to_dev(a)
+
+
+def assert_attn_close(got, ref):
+    np.testing.assert_allclose(got, ref, rtol=RTOL, atol=ATOL)
+    fro = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert fro <= FRO, fro
+
+
+def run_decode_layer_and_compare(L, orc, case, calls=2):
+    from long_context_sparse_02_b200.runtime import LayerOnDevice
+    lay = LayerOnDevice(case, decode=True)
+    q_seq = np.arange(case.T, dtype=np.int32)
+    q_pos = (case.seq_lens - 1).astype(np.int32)
+    pg = orc.Paged(case.seq_lens, case.block_table, 64, case.num_pages)
+    _, idx, out = orc.layer_forward(case.q_idx, case.w, case.k_cache, case.q, case.kv_cache, case.gate, pg, q_seq,
+                                    q_pos, case.K, case.Dv, case.sm_scale)
+    for call in range(calls):  # the second call finds the workspace the first one left
+        lay.forward()
+        torch.cuda.synchronize()
+        assert L.device_error(reset=True) == 0
+        assert np.array_equal(lay.idx.cpu().numpy(), idx), f"call {call}: indices differ"
+        assert_attn_close(lay.out.float().cpu().numpy().astype(np.float64), out)
+    del lay
+    torch.cuda.empty_cache()
+
+
+def test_decode_B8_L131072_full(L, orc):
+    run_decode_layer_and_compare(L, orc, synth.decode_128k(0))
+
+
+def test_decode_B1_L1048576_full(L, orc):
+    run_decode_layer_and_compare(L, orc, synth.decode_1m(0))
+
+
+def test_prefill_T32768_indexer_and_topk_sampled_rows(L, orc):
+    T, HI, DI, K = 32768, 16, 128, 2048
+    ss = np.random.SeedSequence(11).spawn(4)
+    bt, npg = synth.paged_layout(np.random.default_rng(ss[0]), [T])
+    q_idx = synth.dyadic_e4m3(np.random.default_rng(ss[1]), (T, HI, DI))
+    k_cache = synth.dyadic_e4m3(np.random.default_rng(ss[2]), (npg, 64, DI))
+    w = synth.dyadic_weights(np.random.default_rng(ss[3]), (T, HI))
+    seq_lens = np.array([T], np.int32)
+    q_seq = np.zeros(T, np.int32)
+    q_pos = np.arange(T, dtype=np.int32)
+    scores = torch.empty((T, T), dtype=torch.float32, device="cuda")
+    pg = L.paged(dev(seq_lens), dev(bt), npg)
+    L.indexer_scores(dev(q_idx), dev(w), dev(k_cache), pg, dev(q_seq), dev(q_pos), T, scores)
+    row_len = dev(q_pos + 1)
+    idx = L.topk(scores, row_len, K, T)
+    torch.cuda.synchronize()
+    assert L.device_error(reset=True) == 0
+    rows = np.unique(np.r_[[0, 1, 127, 128, 2046, 2047, 2048, 2049, 16383, 16384, T - 2, T - 1],
+                           np.random.default_rng(5).integers(0, T, 36)]).astype(np.int64)
+    opg = orc.Paged(seq_lens, bt, 64, npg)
+    ref = orc.indexer_scores(q_idx[rows], w[rows], k_cache, opg, q_seq[rows], q_pos[rows], ld=T)
+    got = scores[torch.from_numpy(rows).cuda()].cpu().numpy()
+    for i, r in enumerate(rows):
+        n = int(r) + 1
+        assert np.array_equal(got[i, :n].view(np.uint32), ref[i, :n].view(np.uint32)), f"row {r}: scores differ"
+    ref_idx = orc.topk(ref, q_pos[rows] + 1, K)
+    assert np.array_equal(idx[torch.from_numpy(rows).cuda()].cpu().numpy(), ref_idx)
+    del scores, idx
+    torch.cuda.empty_cache()
+
+
+def test_hybrid_B64_dsa_and_swa_full(L, orc):
+    run_decode_layer_and_compare(L, orc, synth.hybrid_dsa(0), calls=1)
+    sw = synth.swa_case(3, synth.hybrid_seq_lens(0))
+    got = L.swa_decode(dev(sw.q), dev(sw.k_ring), dev(sw.v_ring), dev(sw.seq_lens), sw.window, sw.sm_scale)
+    torch.cuda.synchronize()
+    assert L.device_error(reset=True) == 0
+    ref = orc.swa_decode(sw.q, sw.k_ring, sw.v_ring, sw.seq_lens, sw.window, sw.sm_scale)
+    assert_attn_close(got.float().cpu().numpy().astype(np.float64), ref)
