@@ -59,6 +59,31 @@ double orc_bf16_to_f64(uint16_t b)
     return s ? -v : v;
 }
 
+/* The E4M3 code nearest to x, ties to the even mantissa, finite values of
+ * magnitude 448 (the largest finite, S.1111.110) and above giving +-448 --
+ * the "saturate to finite" conversion.  Steps: the exponent e with
+ * 2^e <= |x| < 2^(e+1) (or the subnormal range |x| < 2^-6, quantum 2^-9);
+ * |x| / 2^(e-3) rounded to an integer q in [8, 16]; q = 16 carries into the
+ * next exponent; the code is (e + 7) << 3 | (q - 8).  NaN gives S.1111.111. */
+uint8_t orc_e4m3_from_f64(double x)
+{
+    uint8_t s = signbit(x) ? 0x80 : 0;
+    if (isnan(x)) return s | 0x7F;
+    double a = fabs(x);
+    if (a >= 448.0) return s | 0x7E;
+    if (a < ldexp(1.0, -6)) {
+        double m = nearbyint(a * 512.0);   /* exact: a power-of-two scaling */
+        return s | (uint8_t)(m >= 8.0 ? 0x08 : (int)m);
+    }
+    int E;
+    frexp(a, &E);                          /* a = f * 2^E, 0.5 <= f < 1 */
+    int e = E - 1;
+    double q = nearbyint(ldexp(a, 3 - e)); /* in [8, 16] */
+    if (q >= 16.0) { q = 8.0; ++e; }
+    if (e > 8 || (e == 8 && q > 14.0)) return s | 0x7E;
+    return s | (uint8_t)(((e + 7) << 3) | ((int)q - 8));
+}
+
 /* ---- paged caches ----------------------------------------------------- */
 
 /* Byte/element offset of logical position `pos` of sequence `b` in a cache
@@ -76,6 +101,36 @@ static int64_t orc_row_index(const int32_t *seq_lens, const int32_t *block_table
     int32_t page = block_table[(int64_t)b * max_blocks + lp];
     if (page < 0 || page >= num_pages) return -1;
     return (int64_t)page * page_size + pos % page_size;
+}
+
+/* ---- the step before the layer: appending new tokens to the caches ----
+ * The indexer keys are FP8 ([P1] Key Capabilities: FP8; one scale per
+ * tensor, read here as a multiplier applied before rounding): token j's
+ * indexer key row becomes e4m3(fp32(bf16 k_new[j, d]) * k_scale) -- the
+ * product rounded once, in fp32 -- at logical position tok_pos[j] of
+ * sequence tok_seq[j] of the paged indexer-key cache; its latent row (when
+ * latent_new is given) is stored there unchanged in the latent cache.  A
+ * position outside its sequence or a page outside the cache makes the call
+ * fail (nothing is defined for it). */
+int orc_append_kv(const uint16_t *k_new, float k_scale, const uint16_t *latent_new,
+                  const int32_t *tok_seq, const int32_t *tok_pos, int n,
+                  const int32_t *seq_lens, const int32_t *block_table, int num_seqs,
+                  int max_blocks, int page_size, int num_pages, int DI, int Dqk,
+                  uint8_t *k_cache, uint16_t *kv_cache)
+{
+    for (int j = 0; j < n; ++j) {
+        int64_t r = orc_row_index(seq_lens, block_table, num_seqs, max_blocks, page_size,
+                                  num_pages, tok_seq[j], tok_pos[j]);
+        if (r < 0) return ORC_EBAD;
+        for (int d = 0; d < DI; ++d) {
+            float x = (float)orc_bf16_to_f64(k_new[(int64_t)j * DI + d]) * k_scale;
+            k_cache[r * DI + d] = orc_e4m3_from_f64((double)x);
+        }
+        if (latent_new)
+            for (int d = 0; d < Dqk; ++d)
+                kv_cache[r * Dqk + d] = latent_new[(int64_t)j * Dqk + d];
+    }
+    return 0;
 }
 
 /* ---- stage 1: indexer scores ------------------------------------------ */

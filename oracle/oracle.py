@@ -45,6 +45,10 @@ def _bind(path: str):
     lib.orc_e4m3_to_f64.restype = D
     lib.orc_bf16_to_f64.argtypes = [ctypes.c_uint16]
     lib.orc_bf16_to_f64.restype = D
+    lib.orc_e4m3_from_f64.argtypes = [D]
+    lib.orc_e4m3_from_f64.restype = ctypes.c_uint8
+    lib.orc_append_kv.argtypes = [P, ctypes.c_float, P, P, P, I, P, P, I, I, I, I, I, I, P, P]
+    lib.orc_append_kv.restype = I
     lib.orc_indexer_scores.argtypes = [P, P, P, P, P, I, I, I, I, P, P, I, I, I, P, L]
     lib.orc_topk.argtypes = [P, L, P, I, I, P]
     lib.orc_sparse_attn.argtypes = [P, P, P, P, I, I, I, I, P, P, I, P, D, I, I, I, I, P, P]
@@ -106,6 +110,10 @@ def e4m3_to_f64(code: int) -> float:
 
 def bf16_to_f64(code: int) -> float:
     return _load().orc_bf16_to_f64(int(code))
+
+
+def e4m3_from_f64(x: float) -> int:
+    return int(_load().orc_e4m3_from_f64(float(x)))
 
 
 class Paged:
@@ -203,3 +211,18 @@ def layer_forward(q_idx, w, k_cache, q, kv_cache, gate, pg: Paged, q_seq, q_pos,
                                    float(sm_scale), _p(scores), ld, _p(idx), _p(out))
     _check(rc, "layer_forward")
     return scores, idx, out
+
+
+def append_kv(k_new, k_scale: float, latent_new, tok_seq, tok_pos, pg: Paged, k_cache, kv_cache):
+    """Returns copies of (k_cache, kv_cache) with the new tokens written in."""
+    k_new = _c(k_new, np.uint16)
+    n, DI = k_new.shape
+    k_cache = _c(k_cache, np.uint8).copy()
+    kv_cache = _c(kv_cache, np.uint16).copy()
+    Dqk = kv_cache.shape[-1]
+    lat = None if latent_new is None else _c(latent_new, np.uint16)
+    rc = _load().orc_append_kv(_p(k_new), float(k_scale), None if lat is None else _p(lat),
+                               _p(_c(tok_seq, np.int32)), _p(_c(tok_pos, np.int32)), n, *pg.args(), DI, Dqk,
+                               _p(k_cache), _p(kv_cache))
+    _check(rc, "append_kv")
+    return k_cache, kv_cache

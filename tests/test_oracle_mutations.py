@@ -38,6 +38,12 @@ MUTANTS = {
     "swa_window_short": ("int64_t p0 = L - W > 0 ? L - W : 0;", "int64_t p0 = L - W + 1 > 0 ? L - W + 1 : 0;"),
     "swa_wrong_slot": ("int64_t slot = (p0 + i) % W;\n                const uint16_t *k",
                        "int64_t slot = i % W;\n                const uint16_t *k"),
+    "e4m3_ties_away": ("double q = nearbyint(ldexp(a, 3 - e)); /* in [8, 16] */",
+                       "double q = round(ldexp(a, 3 - e)); /* in [8, 16] */"),
+    "e4m3_no_saturation": ("if (a >= 448.0) return s | 0x7E;", "if (a >= 480.0) return s | 0x7F;"),
+    "append_scale_after_rounding": ("float x = (float)orc_bf16_to_f64(k_new[(int64_t)j * DI + d]) * k_scale;",
+                                    "float x = (float)orc_e4m3_to_f64(orc_e4m3_from_f64(orc_bf16_to_f64("
+                                    "k_new[(int64_t)j * DI + d]))) * k_scale;"),
 }
 
 PIN_TESTS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]

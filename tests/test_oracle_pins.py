@@ -404,3 +404,66 @@ def test_synth_is_deterministic_and_dyadic():
     assert np.array_equal(v, np.round(v)) and np.abs(v).max() <= 4
     assert np.array_equal(a.w * 64, np.round(a.w * 64))
     assert sorted(set(a.block_table.ravel().tolist())) == list(range(a.num_pages))
+
+
+# ---------------------------------------------------------------- the append step (FP8 quantisation)
+
+def _finite_e4m3_codes():
+    return [c for c in range(256) if (c & 0x7F) != 0x7F]
+
+
+def test_e4m3_encoder_round_trips_every_finite_code(orc):
+    for c in _finite_e4m3_codes():
+        assert orc.e4m3_from_f64(orc.e4m3_to_f64(c)) == c, hex(c)
+
+
+def test_e4m3_encoder_rounds_midpoints_to_even_and_neighbours_to_nearest(orc):
+    # every pair of adjacent finite magnitudes, from the definition: the exact
+    # midpoint goes to the code with the even mantissa, anything off it to the
+    # nearer code
+    for c in range(0x00, 0x7E):
+        lo, hi = orc.e4m3_to_f64(c), orc.e4m3_to_f64(c + 1)
+        mid = (lo + hi) / 2
+        even = c if c % 2 == 0 else c + 1
+        for sgn, sbit in ((1.0, 0x00), (-1.0, 0x80)):
+            assert orc.e4m3_from_f64(sgn * mid) == even | sbit, hex(c)
+            assert orc.e4m3_from_f64(sgn * math.nextafter(mid, 0.0)) == c | sbit
+            assert orc.e4m3_from_f64(sgn * math.nextafter(mid, math.inf)) == (c + 1) | sbit
+
+
+def test_e4m3_encoder_matches_torch_within_range_and_saturates_beyond(orc):
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal(200000) * np.exp2(rng.integers(-12, 9, 200000))).astype(np.float32)
+    x = x[np.abs(x) <= 448.0]
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([orc.e4m3_from_f64(float(v)) for v in x], dtype=np.uint8)
+    assert np.array_equal(got, ref)
+    for v, code in ((448.0, 0x7E), (463.99, 0x7E), (464.0, 0x7E), (465.0, 0x7E), (1e30, 0x7E), (-1e30, 0xFE),
+                    (-500.0, 0xFE), (0.0, 0x00), (-0.0, 0x80), (2.0 ** -10, 0x00), (2.0 ** -9, 0x01)):
+        assert orc.e4m3_from_f64(v) == code, v
+
+
+def test_append_places_rows_through_the_block_table_and_scales_before_rounding(orc):
+    rng = np.random.default_rng(8)
+    bt, npg = one_seq_pages(12, page_size=4, rng=rng, spare=2)
+    seq_lens = np.array([12], np.int32)
+    pg = orc.Paged(seq_lens, bt, 4, npg)
+    k_cache = np.full((npg, 4, 8), 0x55, np.uint8)
+    kv_cache = np.full((npg, 4, 6), 0x1234, np.uint16)
+    kf = np.array([[1.0, -1.5, 0.3, 448.0, 600.0, 2.0 ** -10, -0.0, 7.0]] * 3, np.float32) * np.array([[1], [2], [3]],
+                                                                                                     np.float32)
+    k_new = bf16(kf)
+    lat = rng.integers(0, 65536, (3, 6)).astype(np.uint16)
+    pos = np.array([11, 0, 5], np.int32)
+    kc, vc = orc.append_kv(k_new, 0.5, lat, np.zeros(3, np.int32), pos, pg, k_cache, kv_cache)
+    touched = np.zeros((npg, 4), bool)
+    for j, p in enumerate(pos):
+        page, slot = bt[0, p // 4], p % 4
+        touched[page, slot] = True
+        xs = dec_bf16_torch(k_new[j]).astype(np.float32) * np.float32(0.5)
+        expect = torch.from_numpy(np.clip(xs, -448, 448)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        assert np.array_equal(kc[page, slot], expect)
+        assert np.array_equal(vc[page, slot], lat[j])
+    assert (kc[~touched] == 0x55).all() and (vc[~touched] == 0x1234).all()
+    with pytest.raises(ValueError):  # position past the sequence
+        orc.append_kv(k_new[:1], 1.0, lat[:1], np.zeros(1, np.int32), np.array([12], np.int32), pg, k_cache, kv_cache)
