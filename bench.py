@@ -74,6 +74,8 @@ def parse_args(argv=None):
                     help="wall-clock budget of the --impl reference run")
     ap.add_argument("--prefill-only", type=int, default=0, metavar="T",
                     help="time only the prefill indexer at T queries (small cases for profiling)")
+    ap.add_argument("--append-only", action="store_true",
+                    help="time only the append step (dsa_append_kv), for profiling")
     return ap.parse_args(argv)
 
 
@@ -343,6 +345,7 @@ def run_native(args):
         res["e2e"] = e2e_leg(args, lay, flush, stream, _lib)
         if world == 1 and rank == 0:
             res["prefill_indexer"] = prefill_indexer_leg(args, flush)
+            res["append_kv"] = append_leg(args, flush, peaks)
             res["cpu_baseline"], orc_idx, orc_out = cpu_baseline_leg(case)
             got_idx = lay.idx.cpu().numpy()
             got = lay.out.float().cpu().numpy().astype(np.float64)
@@ -419,6 +422,49 @@ def fp8_peak_tflops():
         torch.cuda.synchronize()
         best = min(best, s.elapsed_time(e))
     return 2 * n ** 3 / (best * 1e-3) / 1e12
+
+
+def append_leg(args, flush, peaks):
+    """The step before the layer: dsa_append_kv for a 32768-token prefill chunk
+    (HBM-bound: per token 2*128 + 2*576 bytes read, 128 + 2*576 written) and for
+    one decode step's 8 tokens (latency), into 128K-token paged caches."""
+    import numpy as np
+    import torch
+    from long_context_sparse_02_b200 import _lib, synth
+    from long_context_sparse_02_b200.runtime import to_dev
+    DI, Dqk, L = 128, 576, 131072
+    ss = np.random.SeedSequence(args.seed + 9).spawn(3)
+    bt, npg = synth.paged_layout(np.random.default_rng(ss[0]), [L])
+    pg = _lib.paged(to_dev(np.array([L], np.int32)), to_dev(bt), npg)
+    k_cache = torch.zeros((npg, 64, DI), dtype=torch.uint8, device="cuda")
+    kv_cache = torch.zeros((npg, 64, Dqk), dtype=torch.bfloat16, device="cuda")
+    out = {}
+    for name, n in (("prefill_chunk", 32768), ("decode_step", 8)):
+        k_new = torch.randn((n, DI), device="cuda").to(torch.bfloat16)
+        lat = torch.randn((n, Dqk), device="cuda").to(torch.bfloat16)
+        tok_seq = torch.zeros(n, dtype=torch.int32, device="cuda")
+        tok_pos = torch.arange(L - n, L, dtype=torch.int32, device="cuda")
+        call = lambda: _lib.append_kv(k_new, 1.0, lat, tok_seq, tok_pos, pg, k_cache, kv_cache)  # noqa: E731
+        for _ in range(3):
+            call()
+        us = []
+        for _ in range(20):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            call()
+            e1.record()
+            torch.cuda.synchronize()
+            us.append(e0.elapsed_time(e1) * 1e3)
+        t = statistics.median(us)
+        nbytes = n * (2 * DI + 2 * Dqk + DI + 2 * Dqk)
+        gbs = nbytes / (t * 1e-6) / 1e9
+        out[name] = {"tokens": n, "us": round(t, 2), "bytes": nbytes, "GB/s": round(gbs, 1),
+                     "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    assert _lib.device_error(reset=True) == 0
+    del k_cache, kv_cache
+    torch.cuda.empty_cache()
+    return out
 
 
 def prefill_indexer_leg(args, flush, T=32768, with_peak=True):
@@ -548,5 +594,10 @@ if __name__ == "__main__":
         build.build()
         fl = L2Flush()
         print(json.dumps(prefill_indexer_leg(a, fl, T=a.prefill_only, with_peak=False)))
+    elif a.append_only:
+        from long_context_sparse_02_b200 import build
+        build.build()
+        fl = L2Flush()
+        print(json.dumps(append_leg(a, fl, load_peaks()[0])))
     else:
         run_native(a)

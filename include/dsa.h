@@ -218,6 +218,28 @@ dsa_status dsa_swa_decode(const uint16_t *q, const uint16_t *k_ring,
                           int32_t B, int32_t H, int32_t D, int32_t window,
                           float sm_scale, uint16_t *out, dsa_stream_t stream);
 
+/* ---- the step before the layer: new tokens into the paged caches ---------------
+ * The indexer keys are stored as FP8 ("aiany.app item naive-n0-5-flash", Key
+ * Capabilities: FP8; "Open-Weight Deployment of an Ultra-Large Sparse Model",
+ * §1: FP8/MXFP8 activations; one scale per tensor here).  For each new token
+ * j, at logical position tok_pos[j] of sequence tok_seq[j] (through the block
+ * table; the position must already be counted in seq_lens):
+ *   k_idx_cache row = e4m3(fp32(k_new[j, d]) * k_scale), the product rounded
+ *                     once to the nearest code, ties to the even mantissa,
+ *                     magnitudes of 448 and above saturating to +-448;
+ *   kv_cache row    = latent_new[j, :] unchanged (skipped when latent_new is NULL).
+ *   k_new       device bf16 [n, DI];  latent_new device bf16 [n, Dqk] or NULL
+ *   tok_seq,tok_pos device int32 [n]
+ *   k_idx_cache device e4m3 [num_pages, 64, DI]; kv_cache device bf16 [num_pages, 64, Dqk]
+ * A position outside its sequence, or a page outside [0, num_pages), skips
+ * that token and sets DSA_DEVERR_POSITION / DSA_DEVERR_PAGE.  Tokens must go to
+ * distinct rows.  Supported: DI in {64, 128}; Dqk a multiple of 8, at most 768.  Buffers
+ * 16-byte aligned.  Needs no workspace. */
+dsa_status dsa_append_kv(const uint16_t *k_new, float k_scale, const uint16_t *latent_new,
+                         const int32_t *tok_seq, const int32_t *tok_pos, const dsa_paged *pg,
+                         int32_t n, int32_t DI, int32_t Dqk, uint8_t *k_idx_cache,
+                         uint16_t *kv_cache, dsa_stream_t stream);
+
 /* ---- housekeeping ---------------------------------------------------------------- */
 const char *dsa_status_string(dsa_status s);
 int32_t dsa_abi_version(void);

@@ -78,6 +78,8 @@ lib.dsa_layer_forward.argtypes = [ctypes.POINTER(LayerArgs), P, SZ, P]
 lib.dsa_layer_forward_profiled.restype = ctypes.c_int
 lib.dsa_layer_forward_profiled.argtypes = [ctypes.POINTER(LayerArgs), P, SZ, ctypes.POINTER(P), P]
 lib.dsa_layer_kernel_launches.restype = I32
+lib.dsa_append_kv.restype = ctypes.c_int
+lib.dsa_append_kv.argtypes = [P, F32, P, P, P, ctypes.POINTER(Paged), I32, I32, I32, P, P, P]
 lib.dsa_layer_kernel_launches.argtypes = [ctypes.POINTER(LayerArgs)]
 lib.dsa_swa_decode.restype = ctypes.c_int
 lib.dsa_swa_decode.argtypes = [P, P, P, P, I32, I32, I32, I32, F32, P, P]
@@ -86,7 +88,7 @@ EXPORTS = ["dsa_abi_version", "dsa_status_string", "dsa_device_error", "dsa_inde
            "dsa_topk_workspace_bytes", "dsa_topk", "dsa_topk_static", "dsa_sparse_attn_workspace_bytes",
            "dsa_sparse_attn",
            "dsa_layer_workspace_bytes", "dsa_layer_forward", "dsa_layer_forward_profiled",
-           "dsa_layer_kernel_launches", "dsa_swa_decode"]
+           "dsa_layer_kernel_launches", "dsa_swa_decode", "dsa_append_kv"]
 
 
 def _check(fn: str, status: int):
@@ -222,3 +224,14 @@ def swa_decode(q, k_ring, v_ring, seq_lens, window: int, sm_scale: float, out=No
         _ptr(seq_lens, torch.int32, "seq_lens"), B, H, D, int(window), float(sm_scale),
         _ptr(out, torch.bfloat16, "out"), _stream()))
     return out
+
+
+def append_kv(k_new, k_scale: float, latent_new, tok_seq, tok_pos, pg: Paged, k_cache, kv_cache):
+    """k_new bf16 [n, DI]; latent_new bf16 [n, Dqk] or None; tok_seq/tok_pos int32 [n];
+    k_cache uint8 (e4m3) [pages, 64, DI] and kv_cache bf16 [pages, 64, Dqk], written in place."""
+    n, DI = k_new.shape
+    Dqk = int(kv_cache.shape[-1]) if kv_cache is not None else 0
+    _check("dsa_append_kv", lib.dsa_append_kv(
+        _ptr(k_new, torch.bfloat16, "k_new"), float(k_scale), _ptr(latent_new, torch.bfloat16, "latent_new", True),
+        _ptr(tok_seq, torch.int32, "tok_seq"), _ptr(tok_pos, torch.int32, "tok_pos"), ctypes.byref(pg), n, DI, Dqk,
+        _ptr(k_cache, torch.uint8, "k_cache"), _ptr(kv_cache, torch.bfloat16, "kv_cache", True), _stream()))

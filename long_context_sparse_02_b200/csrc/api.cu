@@ -315,6 +315,20 @@ int32_t dsa_layer_kernel_launches(const dsa_layer_args *a) {
     return 1 + topk_kernel_launches(a->T, a->max_len) + attn_kernel_launches(a->T, a->K, a->Dv);
 }
 
+dsa_status dsa_append_kv(const uint16_t *k_new, float k_scale, const uint16_t *latent_new, const int32_t *tok_seq,
+                         const int32_t *tok_pos, const dsa_paged *pg, int32_t n, int32_t DI, int32_t Dqk,
+                         uint8_t *k_idx_cache, uint16_t *kv_cache, dsa_stream_t stream) {
+    if (n < 0 || !paged_ok(pg) || !isfinite(k_scale)) return DSA_ERR_INVALID_ARG;
+    if ((DI != 64 && DI != 128) || (latent_new && (Dqk < 8 || Dqk % 8 || Dqk > 768))) return DSA_ERR_UNSUPPORTED;
+    if (n == 0) return DSA_OK;
+    if (!k_new || !tok_seq || !tok_pos || !k_idx_cache || (latent_new && !kv_cache)) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(k_idx_cache) || (latent_new && (!aligned16(latent_new) || !aligned16(kv_cache))))
+        return DSA_ERR_INVALID_ARG;
+    AppendArgs a{k_new, latent_new, tok_seq, tok_pos, paged_dev(pg), n, DI, latent_new ? Dqk : 0, k_scale,
+                 k_idx_cache, kv_cache};
+    return launch_append(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 dsa_status dsa_swa_decode(const uint16_t *q, const uint16_t *k_ring, const uint16_t *v_ring, const int32_t *seq_lens,
                           int32_t B, int32_t H, int32_t D, int32_t window, float sm_scale, uint16_t *out,
                           dsa_stream_t stream) {

@@ -111,6 +111,19 @@ struct SwaArgs {
 };
 dsa_status launch_swa(const SwaArgs &a, cudaStream_t st);
 
+// ---- the append step (new tokens into the paged caches) -----------------------------
+struct AppendArgs {
+    const uint16_t *k_new;       // bf16 [n, DI]
+    const uint16_t *latent_new;  // bf16 [n, Dqk] or NULL
+    const int32_t *tok_seq, *tok_pos;
+    PagedDev pg;
+    int32_t n, DI, Dqk;
+    float k_scale;
+    uint8_t *k_cache;
+    uint16_t *kv_cache;
+};
+dsa_status launch_append(const AppendArgs &a, cudaStream_t st);
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace dsa

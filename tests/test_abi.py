@@ -94,5 +94,16 @@ def test_host_side_argument_errors(lib):
     a.pg = ok_pg
     a.T, a.HI, a.DI, a.K, a.H, a.Dqk, a.Dv, a.max_len, a.sm_scale = 3, 16, 128, 128, 8, 64, 64, 100, 0.1
     assert L.dsa_layer_forward(ctypes.byref(a), None, 0, None) == 1
+    # append: unsupported key width, non-finite scale, bad page size, misaligned keys, missing latent cache
+    assert L.dsa_append_kv(P(16), 1.0, None, P(16), P(16), ctypes.byref(ok_pg), 2, 96, 0, P(16), None, None) == 2
+    assert L.dsa_append_kv(P(16), float("nan"), None, P(16), P(16), ctypes.byref(ok_pg), 2, 128, 0, P(16), None,
+                           None) == 1
+    assert L.dsa_append_kv(P(16), 1.0, None, P(16), P(16), ctypes.byref(bad_pg), 2, 128, 0, P(16), None, None) == 1
+    assert L.dsa_append_kv(P(18), 1.0, None, P(16), P(16), ctypes.byref(ok_pg), 2, 128, 0, P(16), None, None) == 1
+    assert L.dsa_append_kv(P(16), 1.0, P(16), P(16), P(16), ctypes.byref(ok_pg), 2, 128, 576, P(16), None,
+                           None) == 1
+    assert L.dsa_append_kv(P(16), 1.0, P(16), P(16), P(16), ctypes.byref(ok_pg), 2, 128, 570, P(16), P(16),
+                           None) == 2
     # zero-sized calls are no-ops
+    assert L.dsa_append_kv(None, 1.0, None, None, None, ctypes.byref(ok_pg), 0, 128, 0, None, None, None) == 0
     assert L.dsa_topk(P(16), 10, P(16), 0, 8, 10, P(16), None, 0, None) == 0

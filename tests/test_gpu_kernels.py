@@ -301,3 +301,54 @@ def test_layer_decode_topk_fallbacks(L, orc):
         assert np.array_equal(lay.idx.cpu().numpy(), idx), call
         assert_attn_close(bf16_to_np(lay.out), out)
     no_device_error(L)
+
+
+# ------------------------------------------------------------------ the append step
+
+@pytest.mark.parametrize("DI,Dqk,n,scale", [(128, 576, 300, 1.0), (128, 576, 8, 0.0625), (64, 64, 1000, 3.0),
+                                            (128, 0, 77, 0.5)], ids=["decode_576_n300", "scaled_n8", "tiny_n1000",
+                                                                     "keys_only"])
+def test_append_kv_bit_exact(L, orc, DI, Dqk, n, scale):
+    """New tokens' keys quantised to e4m3 and latent rows copied into the
+    paged caches: every byte equal to the oracle's, other rows untouched."""
+    rng = np.random.default_rng(n)
+    seq_lens = np.array([3000, 1700, 900], np.int32)
+    bt, npg = synth.paged_layout(rng, seq_lens)
+    # positions: distinct, spread over the sequences
+    tok_seq = rng.integers(0, 3, n).astype(np.int32)
+    tok_pos = np.empty(n, np.int32)
+    for b in range(3):
+        m = tok_seq == b
+        tok_pos[m] = rng.choice(seq_lens[b], m.sum(), replace=False)
+    # keys: a wide dynamic range, exact e4m3 midpoints, saturation, signed zeros and subnormals
+    kf = (rng.standard_normal((n, DI)) * np.exp2(rng.integers(-14, 10, (n, DI)))).astype(np.float32)
+    kf.ravel()[: 6 * DI] = np.resize(np.array([0.0, -0.0, 448.0, 464.0, 1e6, -1e6, 2.0 ** -10, 3 * 2.0 ** -11,
+                                               0.96875, -0.96875, 17.0, 18.0], np.float32), 6 * DI)
+    k_new = synth.f32_to_bf16_bits(kf)
+    k_cache = rng.integers(0, 256, (npg, 64, DI)).astype(np.uint8)
+    Dc = Dqk if Dqk else 8
+    kv_cache = rng.integers(0, 65536, (npg, 64, Dc)).astype(np.uint16)
+    lat = rng.integers(0, 65536, (n, Dc)).astype(np.uint16) if Dqk else None
+    pg = orc.Paged(seq_lens, bt, 64, npg)
+    ref_k, ref_v = orc.append_kv(k_new, scale, lat, tok_seq, tok_pos, pg, k_cache, kv_cache)
+    dk, dv = dev(k_cache), dev(kv_cache)
+    dpg = L.paged(dev(seq_lens), dev(bt), npg)
+    L.append_kv(dev(k_new), scale, None if lat is None else dev(lat), dev(tok_seq), dev(tok_pos), dpg, dk,
+                dv if Dqk else None)
+    no_device_error(L)
+    assert np.array_equal(dk.cpu().numpy(), ref_k)
+    assert np.array_equal(dv.view(torch.int16).cpu().numpy().view(np.uint16), ref_v)
+
+
+def test_append_kv_reports_bad_positions_without_fault(L, orc):
+    seq_lens = np.array([100], np.int32)
+    bt = np.array([[0, 1]], np.int32)
+    pg = L.paged(dev(seq_lens), dev(bt), 2)
+    k_cache = torch.zeros((2, 64, 128), dtype=torch.uint8, device="cuda")
+    k_new = dev(synth.f32_to_bf16_bits(np.ones((2, 128), np.float32)))
+    L.device_error(reset=True)
+    L.append_kv(k_new, 1.0, None, dev(np.array([0, 0], np.int32)), dev(np.array([100, 5], np.int32)), pg,
+                k_cache, None)
+    torch.cuda.synchronize()
+    assert L.device_error(reset=True) == 1  # DSA_DEVERR_POSITION: position 100 is past the sequence
+    assert (k_cache[0, 5] == 0x38).all() and int(k_cache.sum()) == 0x38 * 128  # only the valid token landed
