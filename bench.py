@@ -346,6 +346,7 @@ def run_native(args):
         if world == 1 and rank == 0:
             res["prefill_indexer"] = prefill_indexer_leg(args, flush)
             res["append_kv"] = append_leg(args, flush, peaks)
+            res["mtp_decode"] = mtp_leg(args, flush, case)
             res["cpu_baseline"], orc_idx, orc_out = cpu_baseline_leg(case)
             got_idx = lay.idx.cpu().numpy()
             got = lay.out.float().cpu().numpy().astype(np.float64)
@@ -422,6 +423,41 @@ def fp8_peak_tflops():
         torch.cuda.synchronize()
         best = min(best, s.elapsed_time(e))
     return 2 * n ** 3 / (best * 1e-3) / 1e12
+
+
+def mtp_leg(args, flush, case, n=4, steps=200):
+    """Several query tokens per sequence (draft tokens of speculative
+    decoding): the decode workload's caches, 4 queries per sequence at its
+    last 4 positions, as explicit (sequence, position) queries through
+    dsa_layer_forward.  Same timing rules as the headline."""
+    import numpy as np
+    import torch
+    from long_context_sparse_02_b200 import synth
+    from long_context_sparse_02_b200.runtime import LayerOnDevice
+    B = case.T
+    q_seq = np.repeat(np.arange(B, dtype=np.int32), n)
+    q_pos = case.seq_lens[q_seq] - n + np.tile(np.arange(n, dtype=np.int32), B)
+    mc = synth.with_queries(case, args.seed + 13, q_seq, q_pos, f"mtp_B{B}x{n}_L{int(case.seq_lens.max())}")
+    lay = LayerOnDevice(mc, decode=False)
+    for _ in range(5):
+        flush.zero_()
+        lay.forward()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record()
+        lay.forward()
+        e1.record()
+    torch.cuda.synchronize()
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev)
+    from long_context_sparse_02_b200 import _lib
+    assert _lib.device_error(reset=True) == 0
+    res = {"workload": mc.name, "queries_per_step": mc.T, "us_per_step": round(ms / steps * 1e3, 2),
+           "tokens_per_s": round(mc.T * steps / (ms / 1e3), 1)}
+    del lay
+    torch.cuda.empty_cache()
+    return res
 
 
 def append_leg(args, flush, peaks):

@@ -185,11 +185,12 @@ typedef struct {
     float *lse;                 /* device fp32 [T, H] or NULL */
 } dsa_layer_args;
 
-/* Workspace: (decode) a per-query histogram of the indexer scores, then the
+/* Workspace: (decode, or T <= 64) a per-query histogram of the indexer scores, then the
  * fp32 scores [T, max_len] + top-K scratch (+ idx if idx_out is NULL) +
- * split-K attention partials.  Decode calls leave the histogram region zeroed
- * and take a faster top-K when they find it zeroed, so reusing one workspace
- * (zero-filled once, or simply reused after a first call) across decode calls
+ * split-K attention partials.  Decode calls (and calls with T <= 64, such as
+ * several draft tokens per sequence) leave the histogram region zeroed and
+ * take a faster top-K when they find it zeroed, so reusing one workspace
+ * (zero-filled once, or simply reused after a first call) across such calls
  * is the fast arrangement; any other contents only cost a slower top-K. */
 size_t dsa_layer_workspace_bytes(const dsa_layer_args *a);
 dsa_status dsa_layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes,

@@ -126,11 +126,16 @@ struct LayerWs {
     size_t total;
 };
 
+// The indexer counts the scores by their top key bits for the top-K whenever
+// it runs its few-query kernel: decode, or up to 64 explicit queries (several
+// draft tokens per sequence, as in speculative decoding).
+bool hist_mode(const dsa_layer_args *a) { return a->mode == DSA_MODE_DECODE || a->T <= 64; }
+
 LayerWs carve_layer(const dsa_layer_args *a, void *ws) {
     LayerWs w{};
     uint8_t *p = static_cast<uint8_t *>(ws);
     size_t off = 0;
-    if (a->mode == DSA_MODE_DECODE) {
+    if (hist_mode(a)) {
         w.score_hist = reinterpret_cast<uint32_t *>(p + off);
         off += align_up((size_t)a->T * SCORE_HIST_BINS * 4, 256);
     }
@@ -277,7 +282,7 @@ dsa_status layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes, dsa
     const PagedDev pg = paged_dev(&a->pg);
     const int64_t ld = (int64_t)ld_of(a->max_len);
     IndexerArgs ia{a->q_idx, a->w, a->k_idx_cache, pg, decode ? nullptr : a->q_seq, decode ? nullptr : a->q_pos,
-                   a->T, a->HI, a->DI, a->max_len, lw.scores, ld, decode ? lw.score_hist : nullptr};
+                   a->T, a->HI, a->DI, a->max_len, lw.scores, ld, hist_mode(a) ? lw.score_hist : nullptr};
     if (!mark(0)) return DSA_ERR_CUDA;
     dsa_status s = launch_indexer(ia, st);
     if (s != DSA_OK) return s;
@@ -286,7 +291,7 @@ dsa_status layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes, dsa
                 decode ? (int32_t)ROWLEN_SEQ_LENS : (int32_t)ROWLEN_QPOS_PLUS_1,
                 a->T, a->K, a->max_len, lw.idx, lw.topk_ws, lw.topk_bytes};
     ta.pdl = true;
-    if (decode) ta.hist = lw.score_hist;
+    if (hist_mode(a)) ta.hist = lw.score_hist;
     s = launch_topk(ta, st);
     if (s != DSA_OK) return s;
     if (!mark(2)) return DSA_ERR_CUDA;

@@ -804,7 +804,7 @@ dsa_status launch_indexer(const IndexerArgs &a, cudaStream_t st) {
     if (!dev) return DSA_ERR_CUDA;
     if (a.T == 0) return DSA_OK;
     IdxParams p{a.w, a.q_seq, a.q_pos, a.pg, a.T, a.HI, a.max_len, a.scores, a.ld, dev->err,
-                a.q_seq == nullptr ? a.hist : nullptr};
+                (a.q_seq == nullptr || a.T <= 64) ? a.hist : nullptr};  // the few-query kernel counts
     const CUtensorMapSwizzle swz = a.DI == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUtensorMap km, qm;
     if (!make_tmap_2d(&km, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.DI, (uint64_t)a.pg.num_pages * 64, a.DI,

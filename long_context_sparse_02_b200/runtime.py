@@ -62,5 +62,6 @@ class LayerOnDevice:
     def scores(self) -> torch.Tensor:
         """The fp32 scores the last forward left at the head of the workspace."""
         ld = (self.max_len + 3) // 4 * 4
-        off = (self.case.T * 2048 * 4 + 255) // 256 * 256 if self.decode else 0  # the decode score histogram
+        # the score histogram comes first in decode, or with up to 64 explicit queries
+        off = (self.case.T * 2048 * 4 + 255) // 256 * 256 if (self.decode or self.case.T <= 64) else 0
         return self.ws[off: off + self.case.T * ld * 4].view(torch.float32).view(self.case.T, ld)

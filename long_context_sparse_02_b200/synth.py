@@ -186,6 +186,29 @@ def decode_1m(seed: int = 0) -> LayerCase:
     return decode_case(seed, [1 << 20], HI=32, name="decode_B1_L1048576")
 
 
+def mtp_decode(seed: int = 0, B: int = 8, L: int = 131072, n: int = 4, HI: int = 32) -> LayerCase:
+    """Several query tokens per sequence at its last n positions (draft tokens
+    of speculative decoding), as explicit (sequence, position) queries."""
+    seq_lens = np.full(B, L, np.int32) if np.isscalar(L) else np.asarray(L, np.int32)
+    q_seq = np.repeat(np.arange(B, dtype=np.int32), n)
+    q_pos = (seq_lens[q_seq] - n + np.tile(np.arange(n, dtype=np.int32), B)).astype(np.int32)
+    return layer_case(f"mtp_B{B}x{n}_L{int(seq_lens.max())}", seed, seq_lens, q_seq, q_pos, HI=HI, DI=128, K=2048,
+                      H=128, Dqk=576, Dv=512)
+
+
+def with_queries(case: LayerCase, seed: int, q_seq, q_pos, name: str) -> LayerCase:
+    """The same caches with other (sequence, position) queries: new query-side
+    tensors (indexer queries and weights, attention queries, gate logits) of
+    the case's shapes, one seeded sub-stream each."""
+    q_seq = np.asarray(q_seq, dtype=np.int32)
+    q_pos = np.asarray(q_pos, dtype=np.int32)
+    T = int(q_seq.shape[0])
+    r_qi, r_w, r_q, r_g = [np.random.default_rng(s) for s in np.random.SeedSequence(seed).spawn(4)]
+    return dataclasses.replace(case, name=name, q_idx=dyadic_e4m3(r_qi, (T, case.HI, case.DI)),
+                               w=dyadic_weights(r_w, (T, case.HI)), q=normal_bf16(r_q, (T, case.H, case.Dqk)),
+                               gate=normal_bf16(r_g, (T, case.H)), q_seq=q_seq, q_pos=q_pos)
+
+
 def prefill_case(seed: int, T: int, HI: int = 16, DI: int = 128, K: int = 2048, H: int = 128,
                  Dqk: int = 576, Dv: int = 512, **kw) -> LayerCase:
     """One sequence of T tokens, every token a causal query."""

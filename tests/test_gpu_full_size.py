@@ -7,6 +7,8 @@ The same calls and launch configurations the benchmark times:
   output element compared;
 * decode, one sequence of 1,048,576 tokens (the longest context; its top-K row
   does not fit a cluster's shared memory) -- every index and output compared;
+* four draft tokens per sequence (speculative decoding), 8 x 131072, as 32
+  explicit (sequence, position) queries through dsa_layer_forward;
 * prefill indexer, one sequence of T = 32768 causal queries (16x128) through
   dsa_indexer_scores and dsa_topk over all 32768 rows -- scores and indices of
   sampled rows (the first, last and tile-boundary rows plus seeded random ones)
@@ -74,6 +76,25 @@ def test_decode_B8_L131072_full(L, orc):
 
 def test_decode_B1_L1048576_full(L, orc):
     run_decode_layer_and_compare(L, orc, synth.decode_1m(0))
+
+
+def test_mtp_decode_B8x4_L131072_full(L, orc):
+    """Four draft tokens per sequence (speculative decoding) at 128K: 32
+    explicit (sequence, position) queries through dsa_layer_forward."""
+    from long_context_sparse_02_b200.runtime import LayerOnDevice
+    c = synth.mtp_decode(0)
+    lay = LayerOnDevice(c, decode=False)
+    pg = orc.Paged(c.seq_lens, c.block_table, 64, c.num_pages)
+    _, idx, out = orc.layer_forward(c.q_idx, c.w, c.k_cache, c.q, c.kv_cache, c.gate, pg, c.q_seq, c.q_pos, c.K,
+                                    c.Dv, c.sm_scale)
+    for call in range(2):
+        lay.forward()
+        torch.cuda.synchronize()
+        assert L.device_error(reset=True) == 0
+        assert np.array_equal(lay.idx.cpu().numpy(), idx), f"call {call}: indices differ"
+        assert_attn_close(lay.out.float().cpu().numpy().astype(np.float64), out)
+    del lay
+    torch.cuda.empty_cache()
 
 
 def test_prefill_T32768_indexer_and_topk_sampled_rows(L, orc):

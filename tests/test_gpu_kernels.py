@@ -246,6 +246,7 @@ LAYER_CASES = [
     ("decode_ragged", lambda: synth.decode_case(3, [1, 65, 2048, 2049, 7000], K=2048, HI=32), True),
     ("decode_h16", lambda: synth.decode_case(4, [5000, 12345], K=2048, HI=16), True),
     ("prefill_T300_K128", lambda: synth.prefill_case(5, 300, K=128), False),
+    ("mtp_ragged_3_drafts", lambda: synth.mtp_decode(8, B=4, L=[2050, 9000, 130, 4097], n=3), False),
     ("prefill_two_seqs", lambda: synth.layer_case(
         "two", 6, [200, 300], np.r_[np.zeros(200, np.int32), np.ones(300, np.int32)],
         np.r_[np.arange(200), np.arange(300)].astype(np.int32), HI=16, DI=128, K=128, H=16, Dqk=576, Dv=512), False),
