@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(DecCfg<DI, NH>::THREADS, DecCfg<DI, NH>::CTAS_
     if (p.hist)
         for (int i = threadIdx.x; i < C::EPI_GROUPS * C::HIST_WORDS; i += blockDim.x) hist_sm[i] = 0;
 
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 32) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
@@ -190,29 +190,63 @@ __global__ void __launch_bounds__(DecCfg<DI, NH>::THREADS, DecCfg<DI, NH>::CTAS_
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
-        tstart[0] = 0;
         fence_mbar_init();
         tma_prefetch_desc(&kmap);
         tma_prefetch_desc(&qmap);
     }
     if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
-    for (int t = threadIdx.x; t < T; t += blockDim.x) {
-        QInfo qi = query_info(t, p.q_seq, p.q_pos, p.pg, p.max_len, nullptr);
-        tstart[t + 1] = (qi.last + 1 + 127) >> 7;
-    }
-    __syncthreads();
-    if (warp == 0) {  // inclusive scan of the per-query tile counts
-        int running = 0;
-        for (int base = 0; base < T; base += 32) {
-            const int i = base + lane;
-            int v = i < T ? tstart[i + 1] : 0;
+    // Per-query tile counts -> their inclusive scan tstart -> this CTA's share
+    // [lo, hi) of the flattened (query, tile) space.  With up to 64 queries
+    // warp 0 does it alone and goes on to look up the pages of its first 32
+    // tiles while the other warps set up barriers and TMEM, so the first key
+    // tile is issued right after set-up.
+    const bool early = T <= 64;
+    auto scan_counts = [&](int base, int v, int &running) {  // warp 0: tstart[base+1..] from counts v
+        const int i = base + lane;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                int n = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += n;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int x = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += x;
+        }
+        if (i < T) tstart[i + 1] = running + v;
+        running += __shfl_sync(0xffffffffu, v, 31);
+    };
+    int w0_tq = -1, w0_p0 = -1, w0_p1 = -1;  // early: lane's tile of the producer's first window
+    if (early) {
+        if (warp == 0) {
+            int cnt[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int t = lane + 32 * h;
+                cnt[h] = t < T ? (query_info(t, p.q_seq, p.q_pos, p.pg, p.max_len, nullptr).last + 1 + 127) >> 7 : 0;
             }
-            if (i < T) tstart[i + 1] = running + v;
-            running += __shfl_sync(0xffffffffu, v, 31);
+            if (lane == 0) tstart[0] = 0;
+            int running = 0;
+            scan_counts(0, cnt[0], running);
+            if (T > 32) scan_counts(32, cnt[1], running);
+            __syncwarp();
+            const int64_t tot = tstart[T];
+            const int64_t lo0 = tot * blockIdx.x / gridDim.x, hi0 = tot * (blockIdx.x + 1) / gridDim.x;
+            if (lane < hi0 - lo0) {
+                const int64_t g = lo0 + lane;
+                w0_tq = locate(tstart, T, g);
+                const int j = static_cast<int>(g - tstart[w0_tq]);
+                const QInfo qi = query_info(w0_tq, p.q_seq, p.q_pos, p.pg, p.max_len, p.err);
+                w0_p0 = page_of(p.pg, qi.b, 2 * j, p.err);
+                w0_p1 = (2 * j + 1) * 64 <= qi.last ? page_of(p.pg, qi.b, 2 * j + 1, p.err) : -1;
+            }
+        }
+    } else {
+        for (int t = threadIdx.x; t < T; t += blockDim.x) {
+            QInfo qi = query_info(t, p.q_seq, p.q_pos, p.pg, p.max_len, nullptr);
+            tstart[t + 1] = (qi.last + 1 + 127) >> 7;
+        }
+        if (threadIdx.x == 0) tstart[0] = 0;
+        __syncthreads();
+        if (warp == 0) {
+            int running = 0;
+            for (int base = 0; base < T; base += 32) scan_counts(base, base + lane < T ? tstart[base + lane + 1] : 0,
+                                                                 running);
         }
     }
     tc_fence_before();
@@ -241,8 +275,8 @@ __global__ void __launch_bounds__(DecCfg<DI, NH>::THREADS, DecCfg<DI, NH>::CTAS_
                 p1 = (2 * j + 1) * 64 <= qi.last ? page_of(p.pg, qi.b, 2 * j + 1, p.err) : -1;
             }
         };
-        int tq, p0, p1;
-        lookup(lane, tq, p0, p1);
+        int tq = w0_tq, p0 = w0_p0, p1 = w0_p1;
+        if (!early) lookup(lane, tq, p0, p1);
         // keys are read once: let them leave L2 first, so the scores written
         // meanwhile are still there for the top-K that follows
         const uint64_t kpol = l2_policy_evict_first();
