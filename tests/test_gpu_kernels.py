@@ -60,6 +60,9 @@ INDEXER_CASES = [
     ("decode_h16_d128", 16, 128, [3000, 257], "decode", False),
     ("decode_h64_d64", 64, 64, [70, 2050], "decode", True),
     ("decode_h4_d64", 4, 64, [1500], "decode", False),
+    # few explicit queries, several per sequence: grouped key streams (runs of 5 -> 4 + 1, singletons, a return)
+    ("drafts_h32_d128", 32, 128, [3000, 257, 5000], "drafts", True),
+    ("drafts_h16_d128", 16, 128, [4999, 130, 2050], "drafts", False),
 ]
 
 
@@ -70,6 +73,12 @@ def _indexer_case(HI, DI, seq_lens, kind, signed, seed=7):
         T = seq_lens[0]
         return synth.layer_case("p", seed, seq_lens, np.zeros(T, np.int32), np.arange(T, dtype=np.int32), HI=HI,
                                 DI=DI, K=64, H=1, Dqk=64, Dv=64, w_signed=signed)
+    if kind == "drafts":
+        q_seq = np.array([0, 0, 0, 0, 0, 1, 2, 2, 2, 0, 1], np.int32)
+        last = np.asarray(seq_lens, np.int32)[q_seq] - 1
+        back = np.array([4, 3, 2, 1, 0, 0, 2, 1, 0, 0, 77], np.int32)  # distinct positions, the last ones first
+        return synth.layer_case("d", seed, seq_lens, q_seq, np.maximum(last - back, 0), HI=HI, DI=DI, K=64, H=1,
+                                Dqk=64, Dv=64, w_signed=signed)
     # two sequences, every token of each a query, concatenated
     q_seq = np.concatenate([np.full(n, b, np.int32) for b, n in enumerate(seq_lens)])
     q_pos = np.concatenate([np.arange(n, dtype=np.int32) for n in seq_lens])
