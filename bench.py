@@ -187,6 +187,10 @@ def source_hash(*names):
     return h.hexdigest()[:16]
 
 
+# the files that define the decode indexer kernel (the grouped few-query kernel lives apart)
+INDEXER_SOURCES = ("indexer.cu", "indexer_common.cuh", "dsa_device.cuh")
+
+
 def profiled_traffic():
     """dram read+write bytes per launch of the decode indexer from the committed
     ncu summary, or None when the kernel source changed since that capture."""
@@ -197,7 +201,7 @@ def profiled_traffic():
     t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
     if not m or not t:
         return None, "summary lacks traffic/source hash"
-    if m.group(1) != source_hash("indexer.cu", "dsa_device.cuh"):
+    if m.group(1) != source_hash(*INDEXER_SOURCES):
         return None, "indexer source changed since the ncu capture"
     return float(t.group(1)), "ncu capture (profiles/)"
 

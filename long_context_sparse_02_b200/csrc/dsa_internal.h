@@ -58,6 +58,10 @@ struct IndexerArgs {
 constexpr int SCORE_HIST_BINS = 2048;
 constexpr int SCORE_HIST_SHIFT = 21;
 dsa_status launch_indexer(const IndexerArgs &a, cudaStream_t st);
+// Few explicit queries (T <= 64, 16 or 32 heads x 128): consecutive queries of
+// one sequence share each key tile.  launch_indexer routes them here.
+bool indexer_group_eligible(const IndexerArgs &a);
+dsa_status launch_indexer_group(const IndexerArgs &a, cudaStream_t st);
 
 // ---- top-K ---------------------------------------------------------------------
 enum RowLenMode : int32_t { ROWLEN_ARRAY = 0, ROWLEN_QPOS_PLUS_1 = 1, ROWLEN_SEQ_LENS = 2 };
