@@ -19,6 +19,9 @@
  *        §2.3 (multi-head screening, 32 heads x 128 dim).
  *   [P1] aiany.app item "naive-n0-5-flash", Key Capabilities (5:1 SWA(128)
  *        and DSA hybrid, 16-head indexer, top 2,048, FP8).
+ *   [P4] "Open-Weight Deployment of an Ultra-Large Sparse Model:
+ *        Architecture, Hardware, and Engineering Practices", §1 and §3
+ *        (activations computed in MXFP8).
  *
  * Every function returns 0 on success and a negative code on bad input.
  * OpenMP spreads independent outputs (key positions, heads, rows) over the
@@ -84,6 +87,59 @@ uint8_t orc_e4m3_from_f64(double x)
     return s | (uint8_t)(((e + 7) << 3) | ((int)q - 8));
 }
 
+/* ---- microscaled FP8 (MXFP8) --------------------------------------------
+ * The pages name MXFP8 as the activation format ("Open-Weight Deployment of
+ * an Ultra-Large Sparse Model", §1 and §3) without defining it; the reading
+ * here is the OCP Microscaling (MX) format: a block of 32 consecutive
+ * elements shares one E8M0 scale, and each element is an E4M3 code; an
+ * element's value is its E4M3 value times the block's scale. */
+#define ORC_MX_BLOCK 32
+
+/* E8M0: 8 exponent bits, bias 127, no sign and no mantissa; code c is
+ * 2^(c - 127) for c in [0, 254], and 255 is NaN. */
+double orc_e8m0_to_f64(uint8_t c)
+{
+    if (c == 255) return NAN;
+    return ldexp(1.0, (int)c - 127);
+}
+
+/* One block of n values to MXFP8.  The shared exponent is floor(log2 of the
+ * largest magnitude) minus 8 -- 8 being the exponent of the largest power of
+ * two that E4M3 holds (256) -- so the largest element lands in [256, 512)
+ * before rounding; it is clamped to the scale's range [-127, 127].  A block
+ * of zeros takes code 0.  Each element becomes the E4M3 code nearest to
+ * x / 2^shared (ties to even; magnitudes of 448 and above, which only the
+ * largest elements reach, give +-448).  Non-finite input is rejected. */
+int orc_mx_encode_block(const double *x, int n, uint8_t *codes, uint8_t *scale)
+{
+    double amax = 0.0;
+    for (int i = 0; i < n; ++i) {
+        if (!isfinite(x[i])) return ORC_EBAD;
+        if (fabs(x[i]) > amax) amax = fabs(x[i]);
+    }
+    int shared = -127;
+    if (amax > 0.0) {
+        int E;
+        frexp(amax, &E);                   /* amax = f * 2^E, 0.5 <= f < 1 */
+        shared = (E - 1) - 8;              /* E - 1 = floor(log2 amax) */
+        if (shared < -127) shared = -127;
+        if (shared > 127) shared = 127;
+    }
+    *scale = (uint8_t)(shared + 127);
+    for (int i = 0; i < n; ++i)
+        codes[i] = orc_e4m3_from_f64(ldexp(x[i], -shared)); /* exact scaling */
+    return 0;
+}
+
+/* nblocks consecutive blocks of ORC_MX_BLOCK values. */
+int orc_mx_encode(const double *x, int64_t nblocks, uint8_t *codes, uint8_t *scales)
+{
+    for (int64_t b = 0; b < nblocks; ++b)
+        if (orc_mx_encode_block(x + b * ORC_MX_BLOCK, ORC_MX_BLOCK, codes + b * ORC_MX_BLOCK, scales + b))
+            return ORC_EBAD;
+    return 0;
+}
+
 /* ---- paged caches ----------------------------------------------------- */
 
 /* Byte/element offset of logical position `pos` of sequence `b` in a cache
@@ -133,6 +189,38 @@ int orc_append_kv(const uint16_t *k_new, float k_scale, const uint16_t *latent_n
     return 0;
 }
 
+/* The MXFP8 variant of the append step: each 32-wide block of token j's
+ * bf16 key row becomes one MXFP8 block (orc_mx_encode_block, no other
+ * scale), its codes stored in the token's row of the paged key cache and its
+ * block scales in the same row of the paged scale cache [num_pages,
+ * page_size, DI/32]; the latent row as in orc_append_kv. */
+int orc_append_kv_mx(const uint16_t *k_new, const uint16_t *latent_new,
+                     const int32_t *tok_seq, const int32_t *tok_pos, int n,
+                     const int32_t *seq_lens, const int32_t *block_table, int num_seqs,
+                     int max_blocks, int page_size, int num_pages, int DI, int Dqk,
+                     uint8_t *k_cache, uint8_t *k_scales, uint16_t *kv_cache)
+{
+    if (DI % ORC_MX_BLOCK) return ORC_EBAD;
+    const int nb = DI / ORC_MX_BLOCK;
+    double x[ORC_MX_BLOCK];
+    for (int j = 0; j < n; ++j) {
+        int64_t r = orc_row_index(seq_lens, block_table, num_seqs, max_blocks, page_size,
+                                  num_pages, tok_seq[j], tok_pos[j]);
+        if (r < 0) return ORC_EBAD;
+        for (int blk = 0; blk < nb; ++blk) {
+            for (int i = 0; i < ORC_MX_BLOCK; ++i)
+                x[i] = orc_bf16_to_f64(k_new[(int64_t)j * DI + blk * ORC_MX_BLOCK + i]);
+            if (orc_mx_encode_block(x, ORC_MX_BLOCK, k_cache + r * DI + blk * ORC_MX_BLOCK,
+                                    k_scales + r * nb + blk))
+                return ORC_EBAD;
+        }
+        if (latent_new)
+            for (int d = 0; d < Dqk; ++d)
+                kv_cache[r * Dqk + d] = latent_new[(int64_t)j * Dqk + d];
+    }
+    return 0;
+}
+
 /* ---- stage 1: indexer scores ------------------------------------------ */
 
 /* I[t,s] = sum_h w[t,h] * max(0, sum_d qI[t,h,d] * kI[s,d]) for every
@@ -168,6 +256,53 @@ int orc_indexer_scores(const uint8_t *q_idx, const float *w,
                 double dot = 0.0;
                 for (int d = 0; d < DI; ++d)
                     dot += q[h * DI + d] * orc_e4m3_to_f64(k[d]);
+                double relu = dot > 0.0 ? dot : 0.0;
+                I += (double)w[(int64_t)t * HI + h] * relu;
+            }
+            scores[t * ld + s] = (float)I;
+        }
+    }
+    free(q);
+    return bad ? ORC_EBAD : 0;
+}
+
+/* The indexer score of orc_indexer_scores with MXFP8 operands: each qI
+ * element is its E4M3 value times the scale of its 32-wide block along DI
+ * (q_scales: E8M0 [T,HI,DI/32]), each cached kI element likewise (k_scales:
+ * E8M0 [num_pages,page_size,DI/32], the key cache's row layout); the score
+ * formula, its fp64 sum and the single rounding to fp32 are unchanged. */
+int orc_indexer_scores_mx(const uint8_t *q_idx, const uint8_t *q_scales, const float *w,
+                          const uint8_t *k_cache, const uint8_t *k_scales,
+                          const int32_t *seq_lens, const int32_t *block_table, int num_seqs,
+                          int max_blocks, int page_size, int num_pages, const int32_t *q_seq,
+                          const int32_t *q_pos, int T, int HI, int DI, float *scores, int64_t ld)
+{
+    if (DI % ORC_MX_BLOCK) return ORC_EBAD;
+    const int nb = DI / ORC_MX_BLOCK;
+    int bad = 0;
+    double *q = (double *)malloc(sizeof(double) * (size_t)HI * DI);
+    for (int t = 0; t < T; ++t) {
+        int b = q_seq[t];
+        int64_t p = q_pos[t];
+        if (b < 0 || b >= num_seqs || p < 0 || p >= seq_lens[b] || p >= ld) { bad |= 1; continue; }
+        for (int h = 0; h < HI; ++h)
+            for (int d = 0; d < DI; ++d) {
+                int64_t e = ((int64_t)t * HI + h) * DI + d;
+                int64_t sc = ((int64_t)t * HI + h) * nb + d / ORC_MX_BLOCK;
+                q[h * DI + d] = orc_e4m3_to_f64(q_idx[e]) * orc_e8m0_to_f64(q_scales[sc]);
+            }
+#pragma omp parallel for schedule(static) reduction(| : bad)
+        for (int64_t s = 0; s <= p; ++s) {
+            int64_t r = orc_row_index(seq_lens, block_table, num_seqs, max_blocks,
+                                      page_size, num_pages, b, s);
+            if (r < 0) { bad |= 1; continue; }
+            const uint8_t *k = k_cache + r * DI;
+            const uint8_t *ks = k_scales + r * nb;
+            double I = 0.0;
+            for (int h = 0; h < HI; ++h) {
+                double dot = 0.0;
+                for (int d = 0; d < DI; ++d)
+                    dot += q[h * DI + d] * (orc_e4m3_to_f64(k[d]) * orc_e8m0_to_f64(ks[d / ORC_MX_BLOCK]));
                 double relu = dot > 0.0 ? dot : 0.0;
                 I += (double)w[(int64_t)t * HI + h] * relu;
             }

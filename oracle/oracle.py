@@ -50,6 +50,14 @@ def _bind(path: str):
     lib.orc_append_kv.argtypes = [P, ctypes.c_float, P, P, P, I, P, P, I, I, I, I, I, I, P, P]
     lib.orc_append_kv.restype = I
     lib.orc_indexer_scores.argtypes = [P, P, P, P, P, I, I, I, I, P, P, I, I, I, P, L]
+    lib.orc_e8m0_to_f64.argtypes = [ctypes.c_uint8]
+    lib.orc_e8m0_to_f64.restype = D
+    lib.orc_mx_encode.argtypes = [P, L, P, P]
+    lib.orc_mx_encode.restype = I
+    lib.orc_append_kv_mx.argtypes = [P, P, P, P, I, P, P, I, I, I, I, I, I, P, P, P]
+    lib.orc_append_kv_mx.restype = I
+    lib.orc_indexer_scores_mx.argtypes = [P, P, P, P, P, P, P, I, I, I, I, P, P, I, I, I, P, L]
+    lib.orc_indexer_scores_mx.restype = I
     lib.orc_topk.argtypes = [P, L, P, I, I, P]
     lib.orc_sparse_attn.argtypes = [P, P, P, P, I, I, I, I, P, P, I, P, D, I, I, I, I, P, P]
     lib.orc_swa_decode.argtypes = [P, P, P, P, I, I, I, I, D, P]
@@ -226,3 +234,72 @@ def append_kv(k_new, k_scale: float, latent_new, tok_seq, tok_pos, pg: Paged, k_
                                _p(k_cache), _p(kv_cache))
     _check(rc, "append_kv")
     return k_cache, kv_cache
+
+
+# ---------------------------------------------------------------- MXFP8 (blocks of 32, E8M0 scales)
+
+MX_BLOCK = 32
+
+
+def e8m0_to_f64(code: int) -> float:
+    return _load().orc_e8m0_to_f64(int(code))
+
+
+def mx_encode(x):
+    """x float64 [..., n], n a multiple of 32: (E4M3 codes [..., n], E8M0 scales [..., n/32])."""
+    x = _c(x, np.float64)
+    n = x.shape[-1]
+    if n % MX_BLOCK:
+        raise ValueError("last dimension must be a multiple of 32")
+    codes = np.empty(x.shape, dtype=np.uint8)
+    scales = np.empty(x.shape[:-1] + (n // MX_BLOCK,), dtype=np.uint8)
+    rc = _load().orc_mx_encode(_p(x), x.size // MX_BLOCK, _p(codes), _p(scales))
+    _check(rc, "mx_encode")
+    return codes, scales
+
+
+def mx_decode(codes, scales):
+    """Values of MXFP8 blocks (float64), from the oracle's own decoders."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    scales = np.asarray(scales, dtype=np.uint8)
+    lib = _load()
+    ev = np.array([lib.orc_e4m3_to_f64(c) for c in range(256)])
+    sv = np.array([lib.orc_e8m0_to_f64(c) for c in range(256)])
+    return ev[codes] * np.repeat(sv[scales], MX_BLOCK, axis=-1)
+
+
+def append_kv_mx(k_new, latent_new, tok_seq, tok_pos, pg: Paged, k_cache, k_scales, kv_cache):
+    """Returns copies of (k_cache, k_scales, kv_cache) with the new tokens written in."""
+    k_new = _c(k_new, np.uint16)
+    n, DI = k_new.shape
+    k_cache = _c(k_cache, np.uint8).copy()
+    k_scales = _c(k_scales, np.uint8).copy()
+    kv_cache = _c(kv_cache, np.uint16).copy()
+    Dqk = kv_cache.shape[-1]
+    lat = None if latent_new is None else _c(latent_new, np.uint16)
+    rc = _load().orc_append_kv_mx(_p(k_new), None if lat is None else _p(lat), _p(_c(tok_seq, np.int32)),
+                                  _p(_c(tok_pos, np.int32)), n, *pg.args(), DI, Dqk, _p(k_cache),
+                                  _p(k_scales), _p(kv_cache))
+    _check(rc, "append_kv_mx")
+    return k_cache, k_scales, kv_cache
+
+
+def indexer_scores_mx(q_idx, q_scales, w, k_cache, k_scales, pg: Paged, q_seq, q_pos, ld=None, fill=-np.inf):
+    """MXFP8 indexer scores [T, ld] fp32; q_scales [T, HI, DI/32], k_scales [pages, page_size, DI/32]."""
+    q_idx = _c(q_idx, np.uint8)
+    T, HI, DI = q_idx.shape
+    q_scales = _c(q_scales, np.uint8).reshape(T, HI, DI // MX_BLOCK)
+    w = _c(w, np.float32).reshape(T, HI)
+    k_cache = _c(k_cache, np.uint8)
+    k_scales = _c(k_scales, np.uint8)
+    if k_scales.size * MX_BLOCK != k_cache.size:
+        raise ValueError("k_scales must hold one scale per 32 key elements")
+    q_seq = _c(q_seq, np.int32)
+    q_pos = _c(q_pos, np.int32)
+    if ld is None:
+        ld = int(q_pos.max()) + 1 if T else 1
+    scores = np.full((T, ld), fill, dtype=np.float32)
+    rc = _load().orc_indexer_scores_mx(_p(q_idx), _p(q_scales), _p(w), _p(k_cache), _p(k_scales), *pg.args(),
+                                       _p(q_seq), _p(q_pos), T, HI, DI, _p(scores), ld)
+    _check(rc, "indexer_scores_mx")
+    return scores

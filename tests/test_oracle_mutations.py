@@ -44,6 +44,13 @@ MUTANTS = {
     "append_scale_after_rounding": ("float x = (float)orc_bf16_to_f64(k_new[(int64_t)j * DI + d]) * k_scale;",
                                     "float x = (float)orc_e4m3_to_f64(orc_e4m3_from_f64(orc_bf16_to_f64("
                                     "k_new[(int64_t)j * DI + d]))) * k_scale;"),
+    "mx_emax_off_by_one": ("shared = (E - 1) - 8;", "shared = (E - 1) - 7;"),
+    "mx_low_clamp_wrong": ("if (shared < -127) shared = -127;", "if (shared < -126) shared = -126;"),
+    "mx_q_scale_ignores_head": ("int64_t sc = ((int64_t)t * HI + h) * nb + d / ORC_MX_BLOCK;",
+                                "int64_t sc = (int64_t)t * nb + d / ORC_MX_BLOCK;"),
+    "mx_k_scale_wrong_block": ("orc_e8m0_to_f64(ks[d / ORC_MX_BLOCK])", "orc_e8m0_to_f64(ks[d % nb])"),
+    "mx_k_scale_dropped": ("(orc_e4m3_to_f64(k[d]) * orc_e8m0_to_f64(ks[d / ORC_MX_BLOCK]))", "orc_e4m3_to_f64(k[d])"),
+    "mx_append_scale_row": ("k_scales + r * nb + blk))", "k_scales + (int64_t)j * nb + blk))"),
 }
 
 PIN_TESTS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]

@@ -467,3 +467,153 @@ def test_append_places_rows_through_the_block_table_and_scales_before_rounding(o
     assert (kc[~touched] == 0x55).all() and (vc[~touched] == 0x1234).all()
     with pytest.raises(ValueError):  # position past the sequence
         orc.append_kv(k_new[:1], 1.0, lat[:1], np.zeros(1, np.int32), np.array([12], np.int32), pg, k_cache, kv_cache)
+
+
+# ---------------------------------------------------------------- MXFP8 (32-element blocks sharing an E8M0 scale)
+
+def test_e8m0_decoder_is_a_power_of_two_on_every_code(orc):
+    for c in range(255):
+        assert orc.e8m0_to_f64(c) == math.ldexp(1.0, c - 127), c
+    assert math.isnan(orc.e8m0_to_f64(255))
+
+
+def test_mx_encoder_hand_worked_blocks(orc):
+    with open(os.path.join(GOLDEN, "mxfp8_blocks.json")) as f:
+        blocks = json.load(f)["blocks"]
+    for blk in blocks:
+        x = np.zeros(32)
+        x[:len(blk["values"])] = [float.fromhex(v) for v in blk["values"]]
+        expect = np.zeros(32, np.uint8)
+        expect[:len(blk["codes"])] = blk["codes"]
+        codes, scale = orc.mx_encode(x[None])
+        assert int(scale[0, 0]) == blk["scale"], blk["name"]
+        assert np.array_equal(codes[0], expect), blk["name"]
+
+
+def test_mx_encoder_round_trips_representable_blocks(orc):
+    """A block whose largest magnitude is an E4M3 value in [256, 448] times
+    2^k, all elements E4M3 values times 2^k, comes back exactly, scale 127+k."""
+    rng = np.random.default_rng(21)
+    finite = np.array(_finite_e4m3_codes(), np.uint8)
+    for _ in range(200):
+        codes = rng.choice(finite, 32).astype(np.uint8)
+        codes[rng.integers(32)] = rng.integers(0x78, 0x7F) | (0x80 if rng.random() < 0.5 else 0)
+        k = int(rng.integers(-100, 101))
+        c2, s2 = orc.mx_encode(np.ldexp(dec_e4m3_torch(codes), k)[None])
+        assert int(s2[0, 0]) == 127 + k
+        assert np.array_equal(c2[0], codes)
+
+
+def test_mx_encoder_elements_match_torch_and_the_scale_brackets_the_largest(orc):
+    """Given the chosen scale, every element is torch's E4M3 cast of x / scale
+    (clipped to the largest finite value), and the largest magnitude over the
+    scale lies in [256, 512)."""
+    rng = np.random.default_rng(22)
+    x = (rng.standard_normal((500, 32)) * np.exp2(rng.integers(-30, 30, (500, 1)))).astype(np.float32)
+    x[::7, 5] = 0.0
+    x = x.astype(np.float64)
+    codes, scales = orc.mx_encode(x)
+    sh = scales.astype(np.int64) - 127
+    r = np.abs(x).max(axis=1) * np.exp2(-sh[:, 0])
+    assert np.all((r >= 256.0) & (r < 512.0))
+    y = np.clip(x * np.exp2(-sh), -448.0, 448.0).astype(np.float32)  # exact: a power-of-two scaling of fp32 values
+    ref = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes, ref)
+
+
+def test_mx_encoder_sign_and_power_of_two_invariance(orc):
+    rng = np.random.default_rng(24)
+    x = (rng.standard_normal((200, 32)) * np.exp2(rng.integers(-20, 20, (200, 1)))).astype(np.float32)
+    x = x.astype(np.float64)
+    c, s = orc.mx_encode(x)
+    cn, sn = orc.mx_encode(-x)
+    assert np.array_equal(sn, s) and np.array_equal(cn, c ^ 0x80)
+    for j in (-5, 3, 17):
+        cj, sj = orc.mx_encode(np.ldexp(x, j))
+        assert np.array_equal(cj, c) and np.array_equal(sj.astype(np.int64), s.astype(np.int64) + j)
+
+
+def _mx_operands(rng, shape):
+    """E4M3 elements in {-4..4}/16 and scale codes in [124, 130]: every sum below is exact in fp32."""
+    codes = e4m3(rng.integers(-4, 5, size=shape).astype(np.float32) / 16)
+    scales = rng.integers(124, 131, size=shape[:-1] + (shape[-1] // 32,)).astype(np.uint8)
+    return codes, scales
+
+
+def _mx_values(codes, scales):
+    """Dequantised with library routines: torch's E4M3 cast and ldexp."""
+    return dec_e4m3_torch(codes) * np.repeat(np.ldexp(1.0, scales.astype(np.int64) - 127), 32, axis=-1)
+
+
+def test_mx_indexer_is_relu_matmul_of_the_dequantised_operands_per_head(orc):
+    """One-hot weights pick each head in turn: I = w * max(0, Q_h K^T) on the
+    dequantised operands (a numpy matmul).  Scales differ per head, per
+    32-block and per key row; the cache's unused rows hold NaN scales."""
+    rng = np.random.default_rng(23)
+    T, HI, DI, L, P = 6, 3, 96, 40, 8
+    qc, qs = _mx_operands(rng, (T, HI, DI))
+    kc_rows, ks_rows = _mx_operands(rng, (L, DI))
+    bt, npg = one_seq_pages(L, P, rng, spare=2)
+    kc = scatter_rows(kc_rows, bt, P, npg)
+    ks = scatter_rows(ks_rows, bt, P, npg, fill=255)
+    pg = orc.Paged([L], bt, P, npg)
+    qpos = rng.integers(0, L, T).astype(np.int32)
+    Qd, Kd = _mx_values(qc, qs), _mx_values(kc_rows, ks_rows)
+    for h in range(HI):
+        w = np.zeros((T, HI), np.float32)
+        w[:, h] = 0.75
+        sc = orc.indexer_scores_mx(qc, qs, w, kc, ks, pg, np.zeros(T, np.int32), qpos, ld=L)
+        ref = (0.75 * np.maximum(Qd[:, h, :] @ Kd.T, 0.0)).astype(np.float32)
+        for t in range(T):
+            n = qpos[t] + 1
+            assert np.array_equal(sc[t, :n], ref[t, :n]), (h, t)
+            assert np.all(np.isneginf(sc[t, n:]))
+
+
+def test_mx_indexer_with_unit_scales_is_the_fp8_indexer_and_uniform_scales_shift_it(orc):
+    rng = np.random.default_rng(26)
+    T, HI, DI, L = 5, 4, 64, 30
+    q, k, bt, npg, kc = _rand_indexer(rng, T, HI, DI, L)
+    w = (rng.integers(-64, 65, (T, HI)) / 64).astype(np.float32)
+    pg = orc.Paged([L], bt, 8, npg)
+    qpos = rng.integers(0, L, T).astype(np.int32)
+    z = np.zeros(T, np.int32)
+    ref = orc.indexer_scores(e4m3(q), w, kc, pg, z, qpos, ld=L)
+
+    def mx(qe, ke):
+        return orc.indexer_scores_mx(e4m3(q), np.full((T, HI, DI // 32), 127 + qe, np.uint8), w, kc,
+                                     np.full(kc.shape[:2] + (DI // 32,), 127 + ke, np.uint8), pg, z, qpos, ld=L)
+
+    assert np.array_equal(mx(0, 0).view(np.uint32), ref.view(np.uint32))
+    fin = np.isfinite(ref)
+    assert np.array_equal(mx(2, -5)[fin], np.ldexp(ref[fin], -3))
+
+
+def test_mx_append_places_encoded_blocks_and_scales_through_the_block_table(orc):
+    rng = np.random.default_rng(25)
+    DI, P, L = 64, 4, 12
+    bt, npg = one_seq_pages(L, P, rng, spare=2)
+    pg = orc.Paged(np.array([L], np.int32), bt, P, npg)
+    k_cache = np.full((npg, P, DI), 0x55, np.uint8)
+    k_scales = np.full((npg, P, DI // 32), 0xAA, np.uint8)
+    kv_cache = np.full((npg, P, 6), 0x1234, np.uint16)
+    kf = (rng.standard_normal((3, DI)) * np.exp2(rng.integers(-20, 20, (3, 2)).repeat(32, axis=1))).astype(np.float32)
+    k_new = bf16(kf)
+    lat = rng.integers(0, 65536, (3, 6)).astype(np.uint16)
+    pos = np.array([11, 0, 5], np.int32)
+    kc, ks, vc = orc.append_kv_mx(k_new, lat, np.zeros(3, np.int32), pos, pg, k_cache, k_scales, kv_cache)
+    codes, scales = orc.mx_encode(dec_bf16_torch(k_new))
+    touched = np.zeros((npg, P), bool)
+    for j, p in enumerate(pos):
+        page, slot = bt[0, p // P], p % P
+        touched[page, slot] = True
+        assert np.array_equal(kc[page, slot], codes[j])
+        assert np.array_equal(ks[page, slot], scales[j])
+        assert np.array_equal(vc[page, slot], lat[j])
+    assert (kc[~touched] == 0x55).all() and (ks[~touched] == 0xAA).all() and (vc[~touched] == 0x1234).all()
+    with pytest.raises(ValueError):  # position past the sequence
+        orc.append_kv_mx(k_new[:1], lat[:1], np.zeros(1, np.int32), np.array([12], np.int32), pg, k_cache, k_scales,
+                         kv_cache)
+    with pytest.raises(ValueError):  # a row that is not whole blocks
+        orc.append_kv_mx(k_new[:, :48], None, np.zeros(3, np.int32), pos, pg, k_cache[..., :48],
+                         k_scales[..., :1], kv_cache)
