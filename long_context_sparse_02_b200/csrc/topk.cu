@@ -460,7 +460,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
         constexpr int NSTEP = 4;
         const int per4 = ((m + CT_WARPS - 1) / CT_WARPS + 127) & ~127;
         const int w0 = warp * per4, w1 = min(m, w0 + per4);
-        // uniform across the cluster: judged on the common slice length, not this CTA's m
+        // uniform across the cluster: decided on the common slice length, not this CTA's m
         // (and on the alignment of the score rows, which is common to every slice)
         const bool fits = (((len + CT_WARPS - 1) / CT_WARPS + 127) & ~127) <= NSTEP * 128 &&
                           (reinterpret_cast<uintptr_t>(a.scores) & 15u) == 0 && (a.ld & 3) == 0;

@@ -9,7 +9,7 @@
  * decoders are written here from the bit-format definitions.
  *
  * Sources (web pages on the method; no page prints a formula, so the score,
- * tie rule and gate form are the build's fixed reading of them):
+ * tie rule and gate form below are readings of their prose):
  *   [P2] "Open-Source LLM Architecture Evolution: How Lightweight Sparse
  *        Attention Reshapes Long-Context Modeling Efficiency",
  *        Architecture Breakdown §2 (bullets "Indexer", "Top-K selection",
