@@ -86,7 +86,11 @@ typedef struct {
  *               last token of sequence t (T == num_seqs, q_pos = seq_len-1)
  *   max_len     host bound: every q_pos[t] < max_len <= ld
  *   scores      device fp32 [T, ld]
- * Supported: HI in {4, 8, 16, 32, 64}, DI in {64, 128}.  Needs no workspace. */
+ * Supported: HI in {4, 8, 16, 32, 64}, DI in {64, 128}.  Needs no workspace.
+ * Performance: with explicit queries, T <= 64, DI = 128 and HI in {16, 32}
+ * (several draft tokens per sequence), each run of up to four consecutive
+ * queries of one sequence reads that sequence's keys once, so list a
+ * sequence's queries next to each other.  Results do not depend on the order. */
 dsa_status dsa_indexer_scores(const uint8_t *q_idx, const float *w,
                               const uint8_t *k_idx_cache, const dsa_paged *pg,
                               const int32_t *q_seq, const int32_t *q_pos,
