@@ -357,6 +357,7 @@ def run_native(args):
             res["parity"] = {"idx_bit_exact": bool(np.array_equal(got_idx, orc_idx)),
                              "out_max_abs_err": float(np.abs(got - orc_out).max()),
                              "out_rel_fro_err": float(np.linalg.norm(got - orc_out) / np.linalg.norm(orc_out))}
+            res.update(long_context_leg(args, flush, peaks))
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -460,6 +461,89 @@ def mtp_leg(args, flush, case, n=4, steps=200):
     res = {"workload": mc.name, "queries_per_step": mc.T, "us_per_step": round(ms / steps * 1e3, 2),
            "tokens_per_s": round(mc.T * steps / (ms / 1e3), 1)}
     del lay
+    torch.cuda.empty_cache()
+    return res
+
+
+def long_context_leg(args, flush, peaks, steps=100):
+    """The layer's other decode workloads, timed like the headline (L2 flushed
+    between steps, outside the events): one sequence of 1,048,576 tokens, and
+    the hybrid serving step -- 64 sequences with lengths uniform in [4096,
+    65536] through one DSA layer (16x128 indexer) and five sliding-window
+    layers (64 heads x 128, window 128, each with its own K/V ring).  Each
+    workload's failure is recorded in its own entry."""
+    import torch
+    from long_context_sparse_02_b200 import _lib, synth
+    from long_context_sparse_02_b200.runtime import LayerOnDevice, to_dev
+    hbm = float(peaks["hbm_gbs"])
+
+    def ms_per_step(fn):
+        for _ in range(5):
+            flush.zero_()
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize()
+        for e0, e1 in ev:
+            flush.zero_()
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        return sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
+
+    def hbm_roofline(nbytes, ms):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"bound": "hbm", "algorithmic_bytes_per_step": nbytes, "achieved": round(gbs, 1), "peak": hbm,
+                "unit": "GB/s", "frac": round(gbs / hbm, 4)}
+
+    def device_ok(entry):
+        err = _lib.device_error(reset=True)
+        if err:
+            entry["device_error"] = hex(err)
+        return entry
+
+    res = {}
+    try:
+        c1 = synth.decode_1m(args.seed)
+        lay = LayerOnDevice(c1, decode=True)
+        ms = ms_per_step(lay.forward)
+        res["decode_1m"] = device_ok({"workload": c1.name, "us_per_step": round(ms * 1e3, 2),
+                                      "tokens_per_s": round(c1.T / (ms * 1e-3), 1),
+                                      "roofline": hbm_roofline(decode_bytes(c1)[0], ms)})
+        del lay, c1
+    except Exception as e:  # recorded, not raised: the headline line must still print
+        res["decode_1m"] = {"error": f"{type(e).__name__}: {e}"[:300]}
+    torch.cuda.empty_cache()
+    try:
+        hc = synth.hybrid_dsa(args.seed)
+        lay = LayerOnDevice(hc, decode=True)
+        sw = synth.swa_case(args.seed + 3, hc.seq_lens)
+        q, seq_lens = to_dev(sw.q), to_dev(sw.seq_lens)
+        k0, v0 = to_dev(sw.k_ring), to_dev(sw.v_ring)
+        rings = [(k0, v0)] + [(k0.clone(), v0.clone()) for _ in range(4)]
+        o = torch.empty_like(q)
+
+        def swa(i=0):
+            _lib.swa_decode(q, rings[i][0], rings[i][1], seq_lens, sw.window, sw.sm_scale, out=o)
+
+        def group():
+            lay.forward()
+            for i in range(5):
+                swa(i)
+
+        B, H, D = sw.q.shape
+        swa_bytes = float(B * H * D * 2 * (2 * min(sw.window, int(sw.seq_lens.min())) + 2))
+        dsa_ms, swa_ms, group_ms = ms_per_step(lay.forward), ms_per_step(swa), ms_per_step(group)
+        res["hybrid"] = device_ok({
+            "workload": f"{hc.name} + 5 x swa_B{B}_H{H}_D{D}_W{sw.window}",
+            "dsa_layer": {"us_per_step": round(dsa_ms * 1e3, 2),
+                          "roofline": hbm_roofline(decode_bytes(hc)[0], dsa_ms)},
+            "swa_layer": {"us_per_step": round(swa_ms * 1e3, 2), "roofline": hbm_roofline(swa_bytes, swa_ms)},
+            "group_1_dsa_5_swa": {"us_per_step": round(group_ms * 1e3, 2),
+                                  "tokens_per_s": round(B / (group_ms * 1e-3), 1)}})
+        del lay, rings, k0, v0
+    except Exception as e:
+        res["hybrid"] = {"error": f"{type(e).__name__}: {e}"[:300]}
     torch.cuda.empty_cache()
     return res
 
