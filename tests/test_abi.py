@@ -107,3 +107,36 @@ def test_host_side_argument_errors(lib):
     # zero-sized calls are no-ops
     assert L.dsa_append_kv(None, 1.0, None, None, None, ctypes.byref(ok_pg), 0, 128, 0, None, None, None) == 0
     assert L.dsa_topk(P(16), 10, P(16), 0, 8, 10, P(16), None, 0, None) == 0
+
+
+def test_layer_workspace_follows_the_documented_layout(lib):
+    """dsa_layer_workspace_bytes (host only) adds up the regions dsa.h lists:
+    the per-query score histogram (2048 bins of 4 bytes, in decode and for
+    T <= 64), the fp32 score rows (ld = max_len rounded up to 4), the idx rows
+    when idx_out is NULL, then the top-K and attention scratch; each of the
+    first three regions 256-byte aligned.  runtime.LayerOnDevice.scores reads
+    the score rows behind that histogram region."""
+    from long_context_sparse_02_b200._lib import LayerArgs
+    L = lib.lib
+
+    def ws(mode, T, max_len, idx_out=None, K=2048, H=128, Dv=512):
+        a = LayerArgs()
+        a.mode, a.T, a.max_len, a.K, a.H, a.Dv, a.HI, a.DI, a.Dqk = mode, T, max_len, K, H, Dv, 32, 128, 576
+        a.idx_out = idx_out
+        return L.dsa_layer_workspace_bytes(ctypes.byref(a))
+
+    def up(n):
+        return (n + 255) // 256 * 256
+
+    for T in (1, 8, 64, 65, 300):
+        for mode in (0, 1):
+            for max_len in (1, 1000, 131072):
+                base = ws(mode, T, max_len, idx_out=ctypes.c_void_p(16))
+                assert ws(mode, T, max_len) - base == up(T * 2048 * 4)
+                hist = up(T * 2048 * 4) if (mode == 1 or T <= 64) else 0
+                rows = up(T * ((max_len + 3) // 4 * 4) * 4)
+                scratch = L.dsa_topk_workspace_bytes(T, 2048, max_len) + L.dsa_sparse_attn_workspace_bytes(T, 128,
+                                                                                                          2048, 512)
+                assert base == hist + rows + scratch, (T, mode, max_len)
+    assert ws(1, 65, 1000) - ws(0, 65, 1000) == up(65 * 2048 * 4)
+    assert ws(0, 0, 10) == 0 and ws(0, 4, 0) == 0 and ws(0, 4, 10, K=0) == 0
