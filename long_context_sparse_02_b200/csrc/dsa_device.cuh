@@ -122,17 +122,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
-// Four rows of a 2-D tensor map (box: one row, `x` the first column) into
-// consecutive box-sized slots at dst, with the map's swizzle.
-__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, uint64_t *bar, int32_t x,
-                                            int32_t y0, int32_t y1, int32_t y2, int32_t y3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
-        : "memory");
-}
-
 // An L2 cache policy that evicts the lines it covers first (for data read once).
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t pol;
@@ -167,14 +156,9 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void 
                  : "memory");
 }
 
-// Contiguous shared -> global copy (bulk async group); both addresses 16-byte
-// aligned, bytes % 16 == 0.  The smem must be made visible to the async proxy
-// first (fence_proxy_async_smem after the generic writes).
-__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)),
-                 "r"(bytes)
-                 : "memory");
-}
+// Bulk async groups of shared -> global stores (tma_store_3d above): the
+// shared memory must be made visible to the async proxy first
+// (fence_proxy_async_smem after the generic writes).
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until every committed bulk store has finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read_all() {
@@ -319,14 +303,6 @@ __device__ __forceinline__ uint32_t dsmem_addr(const void *local, uint32_t rank)
 __device__ __forceinline__ uint2 dsmem_ld_v2(uint32_t remote) {
     uint2 v;
     asm volatile("ld.shared::cluster.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(remote) : "memory");
-    return v;
-}
-__device__ __forceinline__ uint4 dsmem_ld_v4(uint32_t remote) {
-    uint4 v;
-    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(remote)
-                 : "memory");
     return v;
 }
 __device__ __forceinline__ void dsmem_st(uint32_t remote, uint32_t v) {
