@@ -348,7 +348,7 @@ def run_native(args):
     if not args.no_extras:
         res["e2e"] = e2e_leg(args, lay, flush, stream, _lib)
         if world == 1 and rank == 0:
-            res["prefill_indexer"] = prefill_indexer_leg(args, flush)
+            res["prefill_indexer"] = prefill_indexer_leg(args, flush, with_topk=True)
             res["append_kv"] = append_leg(args, flush, peaks)
             res["mtp_decode"] = mtp_leg(args, flush, case)
             res["cpu_baseline"], orc_idx, orc_out = cpu_baseline_leg(case)
@@ -591,7 +591,7 @@ def append_leg(args, flush, peaks):
     return out
 
 
-def prefill_indexer_leg(args, flush, T=32768, with_peak=True):
+def prefill_indexer_leg(args, flush, T=32768, with_peak=True, with_topk=False):
     import numpy as np
     import torch
     from long_context_sparse_02_b200 import _lib, synth
@@ -624,12 +624,53 @@ def prefill_indexer_leg(args, flush, T=32768, with_peak=True):
     flops = 2.0 * HI * DI * T * (T + 1) / 2
     peak = fp8_peak_tflops() if with_peak else float("nan")
     tf = flops / (t * 1e-3) / 1e12
+    res = {"workload": f"prefill_T{T}_indexer_{HI}x{DI}", "ms": round(t, 4), "tflops": round(tf, 1),
+           "fp8_peak_tflops": round(peak, 1), "frac": round(tf / peak, 4), "bound": "tensor",
+           "peak_source": "measured in this run: torch._scaled_mm e4m3 8192^3, best of 10",
+           "algorithmic_flops": flops}
+    if with_topk:
+        res["topk"] = prefill_topk_timing(flush, scores, q_pos, T)
     del scores
     torch.cuda.empty_cache()
-    return {"workload": f"prefill_T{T}_indexer_{HI}x{DI}", "ms": round(t, 4), "tflops": round(tf, 1),
-            "fp8_peak_tflops": round(peak, 1), "frac": round(tf / peak, 4), "bound": "tensor",
-            "peak_source": "measured in this run: torch._scaled_mm e4m3 8192^3, best of 10",
-            "algorithmic_flops": flops}
+    return res
+
+
+def prefill_topk_timing(flush, scores, q_pos, T, K=2048, reps=5):
+    """dsa_topk over the T causal rows the prefill indexer just wrote (row t
+    holds t + 1 scores): HBM-bound on the 4 * T(T+1)/2 bytes of scores read
+    plus the T * K * 4 bytes of indices written.  A failure is recorded, not
+    raised."""
+    import torch
+    from long_context_sparse_02_b200 import _lib
+    try:
+        row_len = q_pos + 1
+        idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
+        need = _lib.topk_workspace_bytes(T, K, T)
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+        call = lambda: _lib.topk(scores, row_len, K, T, idx=idx, ws=ws)  # noqa: E731
+        for _ in range(2):
+            call()
+        ms = []
+        for _ in range(reps):
+            flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            call()
+            e.record()
+            torch.cuda.synchronize()
+            ms.append(s.elapsed_time(e))
+        t = statistics.median(ms)
+        nbytes = 4.0 * T * (T + 1) / 2 + 4.0 * T * K
+        peaks, _ = load_peaks()
+        gbs = nbytes / (t * 1e-3) / 1e9
+        out = {"ms": round(t, 4), "algorithmic_bytes": nbytes, "achieved_gbs": round(gbs, 1),
+               "frac_of_hbm": round(gbs / float(peaks["hbm_gbs"]), 4)}
+        err = _lib.device_error(reset=True)
+        if err:
+            out["device_error"] = hex(err)
+        return out
+    except Exception as e:
+        return {"error": f"{type(e).__name__}: {e}"[:300]}
 
 
 def cpu_baseline_leg(case, min_seconds=10.0, max_steps=8):
