@@ -303,3 +303,84 @@ def indexer_scores_mx(q_idx, q_scales, w, k_cache, k_scales, pg: Paged, q_seq, q
                                        _p(q_seq), _p(q_pos), T, HI, DI, _p(scores), ld)
     _check(rc, "indexer_scores_mx")
     return scores
+
+
+# ---------------------------------------------------------------- context-parallel decode (one long sequence, G ranks)
+
+def rank_ranges(seq_len: int, page_size: int, G: int):
+    """Rank r's contiguous range [lo, hi) of a sequence's positions: the
+    sequence's pages dealt out in G runs of ceil(pages / G) whole pages (the
+    last runs may be short or empty)."""
+    pages = -(-int(seq_len) // page_size)
+    per = -(-pages // G) if pages else 0
+    out = []
+    for r in range(G):
+        lo = min(r * per * page_size, seq_len)
+        hi = min((r + 1) * per * page_size, seq_len)
+        out.append((lo, hi))
+    return out
+
+
+def layer_forward_context_parallel(q_idx, w, k_cache, q, kv_cache, gate, pg: Paged, K: int, Dv: int,
+                                   sm_scale: float, G: int):
+    """The decode layer (query b at the last position of sequence b) with
+    every sequence's history split over G ranks by rank_ranges.  Per rank:
+    the indexer scores of its own positions and their top-K (candidate
+    (score, position) pairs).  The union of the G lists, under the top-K's
+    order (score descending, position ascending, -0 equal to +0), cut to K
+    and sorted by position, is the selection -- the same as one device's,
+    because a position among the K best of the whole history is among the K
+    best of its own range.  Per rank: attention over the selected rows it
+    holds, giving (out_r, lse_r); the output is sum_r exp(lse_r - L) out_r
+    with L = logsumexp_r lse_r (the gate, one factor per (token, head), is
+    common to every rank's term).  Returns (idx [B, K], out [B, H, Dv])."""
+    q_idx = _c(q_idx, np.uint8)
+    B = q_idx.shape[0]
+    P = pg.page_size
+    seq_lens = pg.seq_lens
+    assert B == pg.num_seqs
+    cand_s = [[] for _ in range(B)]
+    cand_p = [[] for _ in range(B)]
+    ranges = [rank_ranges(int(seq_lens[b]), P, G) for b in range(B)]
+    locals_ = []
+    for r in range(G):
+        lo = np.array([ranges[b][r][0] for b in range(B)], np.int64)
+        hi = np.array([ranges[b][r][1] for b in range(B)], np.int64)
+        n = (hi - lo).astype(np.int32)
+        # the rank's own block table: the sequences' pages from lo on (lo is page-aligned)
+        bt = np.full(pg.block_table.shape, -1, np.int32)
+        for b in range(B):
+            nb = -(-int(n[b]) // P)
+            bt[b, :nb] = pg.block_table[b, lo[b] // P: lo[b] // P + nb]
+        pr = Paged(n, bt, P, pg.num_pages)
+        locals_.append((lo, hi, pr))
+        live = np.nonzero(n > 0)[0]
+        if len(live) == 0:
+            continue
+        ld = int(n.max())
+        sc = indexer_scores(q_idx[live], _c(w, np.float32)[live], k_cache, pr, live.astype(np.int32),
+                            (n[live] - 1).astype(np.int32), ld=ld)
+        kept = topk(sc, n[live], K)
+        for i, b in enumerate(live):
+            sel = kept[i][kept[i] >= 0]
+            cand_s[b].append(sc[i, sel])
+            cand_p[b].append(sel.astype(np.int64) + lo[b])
+    idx = np.full((B, K), -1, np.int32)
+    for b in range(B):
+        s = np.concatenate(cand_s[b]) if cand_s[b] else np.zeros(0, np.float32)
+        p = np.concatenate(cand_p[b]) if cand_p[b] else np.zeros(0, np.int64)
+        order = np.lexsort((p, -s.astype(np.float64)))[:K]  # score descending, then position ascending
+        keep = np.sort(p[order])
+        idx[b, :len(keep)] = keep
+    H = _c(q, np.uint16).shape[1]
+    outs, lses = [], []
+    for lo, hi, pr in locals_:
+        li = np.where((idx >= lo[:, None]) & (idx < hi[:, None]), idx - lo[:, None], -1).astype(np.int32)
+        o, l = sparse_attn(q, kv_cache, pr, np.arange(B, dtype=np.int32), li, gate, sm_scale, Dv, return_lse=True)
+        outs.append(o)
+        lses.append(l)
+    lse = np.stack(lses)                                    # [G, B, H]
+    m = lse.max(axis=0)
+    wgt = np.where(np.isneginf(lse), 0.0, np.exp(lse - np.where(np.isneginf(m), 0.0, m)))
+    out = (wgt[..., None] * np.stack(outs)).sum(axis=0) / np.maximum(wgt.sum(axis=0), 1e-300)[..., None]
+    return idx, out

@@ -56,25 +56,27 @@ MUTANTS = {
 PIN_TESTS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]
 
 
+def _pin_calls(fn, orc):
+    """The keyword sets pytest would call a pin with: orc, and each value of
+    its (single-argument) parametrize marks."""
+    import inspect
+    base = {"orc": orc} if "orc" in inspect.signature(fn).parameters else {}
+    calls = [base]
+    for mark in getattr(fn, "pytestmark", []):
+        if mark.name == "parametrize":
+            name, values = mark.args[0], mark.args[1]
+            calls = [dict(c, **{name: v}) for c in calls for v in values]
+    return calls
+
+
 def _pin_failures(orc):
     failed = []
     for fn in PIN_TESTS:
-        args = {}
-        import inspect
-        params = inspect.signature(fn).parameters
-        if "orc" in params:
-            args["orc"] = orc
-        if "kind" in params:
-            for kind in ("normal", "ties", "zeros", "const", "dyadic"):
-                try:
-                    fn(orc=orc, kind=kind)
-                except Exception:
-                    failed.append(f"{fn.__name__}[{kind}]")
-            continue
-        try:
-            fn(**args)
-        except Exception:
-            failed.append(fn.__name__)
+        for kw in _pin_calls(fn, orc):
+            try:
+                fn(**kw)
+            except Exception:
+                failed.append(f"{fn.__name__}{sorted((k, v) for k, v in kw.items() if k != 'orc')}")
     return failed
 
 
@@ -96,3 +98,52 @@ def test_planted_mistake_is_caught(orc, name):
 
 def test_unmutated_oracle_passes_every_pin(orc):
     assert _pin_failures(orc) == []
+
+
+# ---- the context-parallel decode oracle (Python): planted in a copy of oracle.py
+
+PY_SRC = os.path.join(os.path.dirname(SRC), "oracle.py")
+
+PY_MUTANTS = {
+    "cp_ties_to_higher_position": ("order = np.lexsort((p, -s.astype(np.float64)))[:K]",
+                                   "order = np.lexsort((-p, -s.astype(np.float64)))[:K]"),
+    "cp_merge_unweighted": ("out = (wgt[..., None] * np.stack(outs)).sum(axis=0)",
+                            "out = (np.stack(outs) * (wgt[..., None] > 0)).sum(axis=0)"),
+    "cp_local_positions_not_offset": ("cand_p[b].append(sel.astype(np.int64) + lo[b])",
+                                      "cand_p[b].append(sel.astype(np.int64))"),
+    "cp_rank_misses_its_last_position": ("(n[live] - 1).astype(np.int32), ld=ld)",
+                                         "np.maximum(n[live] - 2, 0).astype(np.int32), ld=ld)"),
+}
+
+
+def _cp_pin_failures(mod):
+    runs = [(pins.test_context_parallel_decode_is_the_single_device_layer, {}),
+            (pins.test_context_parallel_decode_breaks_threshold_ties_across_ranks_by_position, {"w_sign": 1.0}),
+            (pins.test_context_parallel_decode_breaks_threshold_ties_across_ranks_by_position, {"w_sign": -1.0})]
+    failed = []
+    for fn, kw in runs:
+        try:
+            fn(orc=mod, **kw)
+        except Exception:
+            failed.append(fn.__name__)
+    return failed
+
+
+def _py_module(src):
+    import types
+    mod = types.ModuleType("oracle_variant")
+    mod.__file__ = PY_SRC
+    exec(compile(src, PY_SRC, "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_planted_mistake_in_the_context_parallel_oracle_is_caught(name):
+    old, new = PY_MUTANTS[name]
+    src = open(PY_SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found"
+    assert _cp_pin_failures(_py_module(src.replace(old, new, 1))), f"no pin caught '{name}'"
+
+
+def test_unmutated_context_parallel_oracle_passes_its_pins():
+    assert _cp_pin_failures(_py_module(open(PY_SRC).read())) == []

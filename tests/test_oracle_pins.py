@@ -617,3 +617,66 @@ def test_mx_append_places_encoded_blocks_and_scales_through_the_block_table(orc)
     with pytest.raises(ValueError):  # a row that is not whole blocks
         orc.append_kv_mx(k_new[:, :48], None, np.zeros(3, np.int32), pos, pg, k_cache[..., :48],
                          k_scales[..., :1], kv_cache)
+
+
+# ---------------------------------------------------------------- context-parallel decode (one long sequence over G ranks)
+
+def _decode_ref(orc, c):
+    pg = orc.Paged(c.seq_lens, c.block_table, c.page_size, c.num_pages)
+    B = len(c.seq_lens)
+    _, idx, out = orc.layer_forward(c.q_idx, c.w, c.k_cache, c.q, c.kv_cache, c.gate, pg,
+                                    np.arange(B, dtype=np.int32), (c.seq_lens - 1).astype(np.int32), c.K, c.Dv,
+                                    c.sm_scale)
+    return pg, idx, out
+
+
+def test_context_parallel_decode_is_the_single_device_layer(orc):
+    """Splitting each sequence's history over G ranks (local top-K, union cut
+    to K, per-rank attention merged by log-sum-exp weights) reproduces the
+    one-device layer: indices exactly, outputs to fp64 rounding.  G = 40
+    leaves most ranks of the short sequences empty."""
+    c = synth.decode_case(5, [700, 130, 2050], HI=4, DI=64, K=64, H=4, Dqk=64, Dv=64)
+    pg, idx, out = _decode_ref(orc, c)
+    for G in (1, 2, 3, 5, 40):
+        got_idx, got = orc.layer_forward_context_parallel(c.q_idx, c.w, c.k_cache, c.q, c.kv_cache, c.gate, pg, c.K,
+                                                          c.Dv, c.sm_scale, G)
+        assert np.array_equal(got_idx, idx), G
+        np.testing.assert_allclose(got, out, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("w_sign", [1.0, -1.0])
+def test_context_parallel_decode_breaks_threshold_ties_across_ranks_by_position(orc, w_sign):
+    """Every key row is one of three rows, so each query's scores take at
+    most three values and the K-th best is shared by positions in several
+    ranks: the union must keep the lowest of them, as one device does.  With
+    negative weights every score is -0.0 or +0.0 or below."""
+    c = synth.decode_case(9, [3000, 1300], HI=4, DI=64, K=64, H=4, Dqk=64, Dv=64)
+    rng = np.random.default_rng(9)
+    distinct = c.k_cache.reshape(-1, c.k_cache.shape[-1])[:3].copy()
+    pick = rng.integers(0, 3, size=c.k_cache.shape[:2])
+    c.k_cache = distinct[pick]
+    c.w = (np.abs(c.w) * w_sign).astype(np.float32)
+    pg, idx, out = _decode_ref(orc, c)
+    sc = orc.indexer_scores(c.q_idx, c.w, c.k_cache, pg, np.arange(2, dtype=np.int32),
+                            (c.seq_lens - 1).astype(np.int32))
+    spans = []
+    for G in (2, 3, 7):
+        got_idx, got = orc.layer_forward_context_parallel(c.q_idx, c.w, c.k_cache, c.q, c.kv_cache, c.gate, pg, c.K,
+                                                          c.Dv, c.sm_scale, G)
+        assert np.array_equal(got_idx, idx), G
+        np.testing.assert_allclose(got, out, rtol=1e-12, atol=1e-13)
+        for b in range(2):
+            row = sc[b, :c.seq_lens[b]]
+            kth = np.sort(row)[::-1][c.K - 1]
+            rr = orc.rank_ranges(int(c.seq_lens[b]), c.page_size, G)
+            spans.append(len({r for p in np.nonzero(row == kth)[0] for r, (lo, hi) in enumerate(rr) if lo <= p < hi}))
+    assert max(spans) >= 2  # the case does put threshold ties in several ranks
+
+
+def test_rank_ranges_cover_the_sequence_in_whole_pages(orc):
+    for L, G in ((700, 3), (130, 5), (64, 2), (1, 4), (0, 2), (1 << 20, 8)):
+        rr = orc.rank_ranges(L, 64, G)
+        assert len(rr) == G and rr[0][0] == 0 and rr[-1][1] == L
+        for (lo, hi), (lo2, _) in zip(rr, rr[1:]):
+            assert lo <= hi == lo2
+        assert all(lo % 64 == 0 for lo, hi in rr if hi > lo)  # a non-empty range starts on a page
