@@ -39,10 +39,6 @@ def f32_to_e4m3_bits(x: np.ndarray) -> np.ndarray:
     return t.view(torch.uint8).numpy()
 
 
-def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
-    return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
-
-
 # ---- building blocks -------------------------------------------------------
 
 def dyadic_e4m3(rng: np.random.Generator, shape, lo: int = -4, hi: int = 4) -> np.ndarray:
