@@ -224,6 +224,24 @@ def decode_bytes(case):
     return layer, indexer
 
 
+def swa_bytes(B, H, D, window, min_len):
+    """Bytes one sliding-window decode layer must move: each sequence's K and
+    V rings over the window (all of it once the sequence is that long), the
+    query row and the output row, bf16."""
+    return float(B * H * D * 2 * (2 * min(window, int(min_len)) + 2))
+
+
+def prefill_topk_bytes(T, K):
+    """The top-K over T causal score rows (row t holds t + 1 fp32 scores):
+    the scores read plus the T x K int32 indices written."""
+    return 4.0 * T * (T + 1) / 2 + 4.0 * T * K
+
+
+def prefill_indexer_flops(T, HI, DI):
+    """2 * HI * DI multiply-adds per (query, causal key) pair, T(T+1)/2 pairs."""
+    return 2.0 * HI * DI * T * (T + 1) / 2
+
+
 # ---------------------------------------------------------------- native arm
 
 def run_native(args):
@@ -532,13 +550,13 @@ def long_context_leg(args, flush, peaks, steps=100):
                 swa(i)
 
         B, H, D = sw.q.shape
-        swa_bytes = float(B * H * D * 2 * (2 * min(sw.window, int(sw.seq_lens.min())) + 2))
+        nbytes_swa = swa_bytes(B, H, D, sw.window, sw.seq_lens.min())
         dsa_ms, swa_ms, group_ms = ms_per_step(lay.forward), ms_per_step(swa), ms_per_step(group)
         res["hybrid"] = device_ok({
             "workload": f"{hc.name} + 5 x swa_B{B}_H{H}_D{D}_W{sw.window}",
             "dsa_layer": {"us_per_step": round(dsa_ms * 1e3, 2),
                           "roofline": hbm_roofline(decode_bytes(hc)[0], dsa_ms)},
-            "swa_layer": {"us_per_step": round(swa_ms * 1e3, 2), "roofline": hbm_roofline(swa_bytes, swa_ms)},
+            "swa_layer": {"us_per_step": round(swa_ms * 1e3, 2), "roofline": hbm_roofline(nbytes_swa, swa_ms)},
             "group_1_dsa_5_swa": {"us_per_step": round(group_ms * 1e3, 2),
                                   "tokens_per_s": round(B / (group_ms * 1e-3), 1)}})
         del lay, rings, k0, v0
@@ -621,7 +639,7 @@ def prefill_indexer_leg(args, flush, T=32768, with_peak=True, with_topk=False):
         torch.cuda.synchronize()
         ms.append(s.elapsed_time(e))
     t = statistics.median(ms)
-    flops = 2.0 * HI * DI * T * (T + 1) / 2
+    flops = prefill_indexer_flops(T, HI, DI)
     peak = fp8_peak_tflops() if with_peak else float("nan")
     tf = flops / (t * 1e-3) / 1e12
     res = {"workload": f"prefill_T{T}_indexer_{HI}x{DI}", "ms": round(t, 4), "tflops": round(tf, 1),
@@ -660,7 +678,7 @@ def prefill_topk_timing(flush, scores, q_pos, T, K=2048, reps=5):
             torch.cuda.synchronize()
             ms.append(s.elapsed_time(e))
         t = statistics.median(ms)
-        nbytes = 4.0 * T * (T + 1) / 2 + 4.0 * T * K
+        nbytes = prefill_topk_bytes(T, K)
         peaks, _ = load_peaks()
         gbs = nbytes / (t * 1e-3) / 1e9
         out = {"ms": round(t, 4), "algorithmic_bytes": nbytes, "achieved_gbs": round(gbs, 1),
