@@ -175,9 +175,19 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": names,
                 "samples": len(self.samples)}
 
+    # reasons that explain clocks below the maximum (a power cap is kept and noted)
+    EXPLAINED = {"sw_power_cap", "hw_power_brake_slowdown", "sync_boost", "applications_clocks_setting"}
+    LOW_FRACTION = 0.85
+
     def rejected(self):
+        """A thermal or hardware slowdown, or SM clocks well below the maximum
+        with no reason that explains them (a leftover clock lock)."""
         s = self.summary()
-        return bool(set(s.get("reasons", [])) & self.BAD)
+        reasons = set(s.get("reasons", []))
+        if reasons & self.BAD:
+            return True
+        mhz, top = s.get("sm_mhz"), s.get("sm_max_mhz")
+        return bool(mhz and top and mhz < self.LOW_FRACTION * top and not reasons & self.EXPLAINED)
 
 
 def source_hash(*names):

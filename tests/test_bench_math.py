@@ -42,3 +42,20 @@ def test_swa_layer_bytes():
 def test_prefill_indexer_flops_and_topk_bytes():
     assert bench.prefill_indexer_flops(32768, 16, 128) == 2_199_090_364_416  # about 2.199e12
     assert bench.prefill_topk_bytes(32768, 2048) == 2_147_549_184 + 268_435_456
+
+
+def _sampler(samples, max_mhz=1965):
+    c = bench.ClockSampler.__new__(bench.ClockSampler)
+    c.ok, c.samples, c.max_mhz = True, samples, max_mhz
+    return c
+
+
+def test_clock_record_rejects_slowdowns_and_unexplained_low_clocks():
+    full, cap, hw, therm = 0, 0x4, 0x8, 0x40
+    assert not _sampler([(1965, full)] * 10).rejected()
+    assert not _sampler([(1300, cap)] * 10).rejected()          # power-capped: kept and noted
+    assert _sampler([(1965, full)] * 9 + [(1965, hw)]).rejected()  # any hardware slowdown
+    assert _sampler([(1800, therm)] * 10).rejected()
+    assert _sampler([(1200, full)] * 10).rejected()              # stuck low with no reason: a clock lock
+    s = _sampler([(1965, full)] * 6 + [(1300, cap)] * 4).summary()
+    assert s["sm_mhz"] == 1965 and s["reasons"] == ["sw_power_cap"] and s["samples"] == 10
