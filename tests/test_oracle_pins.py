@@ -635,13 +635,15 @@ def test_context_parallel_decode_is_the_single_device_layer(orc):
     to K, per-rank attention merged by log-sum-exp weights) reproduces the
     one-device layer: indices exactly, outputs to fp64 rounding.  G = 40
     leaves most ranks of the short sequences empty."""
-    c = synth.decode_case(5, [700, 130, 2050], HI=4, DI=64, K=64, H=4, Dqk=64, Dv=64)
-    pg, idx, out = _decode_ref(orc, c)
-    for G in (1, 2, 3, 5, 40):
-        got_idx, got = orc.layer_forward_context_parallel(c.q_idx, c.w, c.k_cache, c.q, c.kv_cache, c.gate, pg, c.K,
-                                                          c.Dv, c.sm_scale, G)
-        assert np.array_equal(got_idx, idx), G
-        np.testing.assert_allclose(got, out, rtol=1e-12, atol=1e-13)
+    for lens in ([700, 130, 2050], [40, 700]):  # the 40-token sequence is shorter than K: all of it is kept
+        c = synth.decode_case(5, lens, HI=4, DI=64, K=64, H=4, Dqk=64, Dv=64)
+        pg, idx, out = _decode_ref(orc, c)
+        for G in (1, 2, 3, 5, 40):
+            got_idx, got = orc.layer_forward_context_parallel(c.q_idx, c.w, c.k_cache, c.q, c.kv_cache, c.gate, pg,
+                                                              c.K, c.Dv, c.sm_scale, G)
+            assert np.array_equal(got_idx, idx), (lens, G)
+            np.testing.assert_allclose(got, out, rtol=1e-12, atol=1e-13)
+    assert np.array_equal(idx[0, :40], np.arange(40)) and (idx[0, 40:] == -1).all()
 
 
 @pytest.mark.parametrize("w_sign", [1.0, -1.0])
