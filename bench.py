@@ -234,6 +234,11 @@ def decode_bytes(case):
     return layer, indexer
 
 
+# nominal B200 peaks, reported beside the measured ones: HBM3e 7.7 TB/s (HGX), dense FP8 4.5 PFLOP/s
+SPEC_HBM_GBS = 7700.0
+SPEC_FP8_TFLOPS = 4500.0
+
+
 def swa_bytes(B, H, D, window, min_len):
     """Bytes one sliding-window decode layer must move: each sequence's K and
     V rings over the window (all of it once the sequence is that long), the
@@ -344,6 +349,7 @@ def run_native(args):
     traffic, traffic_src = profiled_traffic()
     roofline = {"bound": "hbm", "kernel": "indexer_decode_kernel<128,32> (stage 1 of dsa_layer_forward)",
                 "achieved": round(idx_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(idx_gbs / hbm, 4),
+                "peak_spec": SPEC_HBM_GBS, "frac_spec": round(idx_gbs / SPEC_HBM_GBS, 4),
                 "traffic": traffic, "traffic_source": traffic_src,
                 "algorithmic_bytes_per_launch": idx_bytes, "launch_us": round(st["indexer"], 2),
                 "peak_source": f"hbm_gbs, {peak_src}"}
@@ -364,7 +370,8 @@ def run_native(args):
         "roofline": roofline,
         "layer_roofline": {"bound": "hbm", "algorithmic_bytes_per_step": layer_bytes,
                            "achieved": round(layer_gbs, 1), "peak": hbm, "unit": "GB/s",
-                           "frac": round(layer_gbs / hbm, 4)},
+                           "frac": round(layer_gbs / hbm, 4), "peak_spec": SPEC_HBM_GBS,
+                           "frac_spec": round(layer_gbs / SPEC_HBM_GBS, 4)},
         "stages_us": {k: round(v, 2) for k, v in st.items()},
         "stages_note": f"separate steps with an event between stages (no overlap of kernel boundaries; "
                        f"{st_total:.2f} us per step there)",
@@ -522,7 +529,8 @@ def long_context_leg(args, flush, peaks, steps=100):
     def hbm_roofline(nbytes, ms):
         gbs = nbytes / (ms * 1e-3) / 1e9
         return {"bound": "hbm", "algorithmic_bytes_per_step": nbytes, "achieved": round(gbs, 1), "peak": hbm,
-                "unit": "GB/s", "frac": round(gbs / hbm, 4)}
+                "unit": "GB/s", "frac": round(gbs / hbm, 4), "peak_spec": SPEC_HBM_GBS,
+                "frac_spec": round(gbs / SPEC_HBM_GBS, 4)}
 
     def device_ok(entry):
         err = _lib.device_error(reset=True)
@@ -654,6 +662,7 @@ def prefill_indexer_leg(args, flush, T=32768, with_peak=True, with_topk=False):
     tf = flops / (t * 1e-3) / 1e12
     res = {"workload": f"prefill_T{T}_indexer_{HI}x{DI}", "ms": round(t, 4), "tflops": round(tf, 1),
            "fp8_peak_tflops": round(peak, 1), "frac": round(tf / peak, 4), "bound": "tensor",
+           "fp8_spec_tflops": SPEC_FP8_TFLOPS, "frac_spec": round(tf / SPEC_FP8_TFLOPS, 4),
            "peak_source": "measured in this run: torch._scaled_mm e4m3 8192^3, best of 10",
            "algorithmic_flops": flops}
     if with_topk:

@@ -59,3 +59,7 @@ def test_clock_record_rejects_slowdowns_and_unexplained_low_clocks():
     assert _sampler([(1200, full)] * 10).rejected()              # stuck low with no reason: a clock lock
     s = _sampler([(1965, full)] * 6 + [(1300, cap)] * 4).summary()
     assert s["sm_mhz"] == 1965 and s["reasons"] == ["sw_power_cap"] and s["samples"] == 10
+
+
+def test_nominal_peaks_reported_beside_the_measured_ones():
+    assert bench.SPEC_HBM_GBS == 7700.0 and bench.SPEC_FP8_TFLOPS == 4500.0
