@@ -710,6 +710,23 @@ def prefill_topk_timing(flush, scores, q_pos, T, K=2048, reps=5):
         return {"error": f"{type(e).__name__}: {e}"[:300]}
 
 
+def host_cpu():
+    """The host's CPU model and logical CPU count, recorded beside a CPU timing."""
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    if not model:
+        import platform
+        model = platform.processor() or platform.machine()
+    return {"cpu_model": model, "host_cpus": os.cpu_count()}
+
+
 def cpu_baseline_leg(case, min_seconds=10.0, max_steps=8):
     """The oracle as it stands on this host: whole decode steps of the workload
     (every sequence, full context, all heads), repeated until about
@@ -728,7 +745,7 @@ def cpu_baseline_leg(case, min_seconds=10.0, max_steps=8):
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     cores = int(os.environ.get("OMP_NUM_THREADS", cores))
     return ({"value": round(steps * case.T / dt, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
-             "seconds": round(dt, 2),
+             "seconds": round(dt, 2), **host_cpu(),
              "sample": f"{steps} full decode steps of {case.name} ({case.T} sequences x {case.max_len} tokens, "
                        f"all heads) through oracle.c (fp64, OpenMP)"}, idx, out)
 
@@ -781,7 +798,7 @@ def run_reference(args):
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
            "config": {"workload": f"decode_B{B}_L{Lctx}", "batch_per_gpu": B, "context": Lctx},
            "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": cores, "kind": "oracle",
-                            "sample": sample_desc},
+                            "sample": sample_desc, **host_cpu()},
            "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(res), flush=True)
 
