@@ -406,6 +406,24 @@ def test_synth_is_deterministic_and_dyadic():
     assert sorted(set(a.block_table.ravel().tolist())) == list(range(a.num_pages))
 
 
+def test_draft_query_inputs_follow_their_recipe():
+    """Speculative-decoding queries: the last n positions of each sequence, in
+    sequence order; with_queries keeps the caches and draws new dyadic query
+    tensors, the same for the same seed."""
+    c = synth.mtp_decode(0, B=3, L=[500, 90, 1300], n=4, HI=8)
+    assert np.array_equal(c.q_seq, np.repeat(np.arange(3), 4))
+    assert np.array_equal(c.q_pos, np.concatenate([np.arange(L - 4, L) for L in (500, 90, 1300)]))
+    d = synth.with_queries(c, 7, c.q_seq[::-1].copy(), c.q_pos[::-1].copy(), "reversed")
+    e = synth.with_queries(c, 7, c.q_seq[::-1].copy(), c.q_pos[::-1].copy(), "reversed")
+    for f in ("k_cache", "kv_cache", "block_table", "seq_lens"):
+        assert getattr(d, f) is getattr(c, f)
+    for f in ("q_idx", "w", "q", "gate"):
+        assert np.array_equal(getattr(d, f), getattr(e, f)) and getattr(d, f).shape == getattr(c, f).shape
+    v = dec_e4m3_torch(d.q_idx) * 16
+    assert np.array_equal(v, np.round(v)) and np.abs(v).max() <= 4
+    assert np.array_equal(d.w * 64, np.round(d.w * 64)) and d.w.min() >= 0
+
+
 # ---------------------------------------------------------------- the append step (FP8 quantisation)
 
 def _finite_e4m3_codes():
