@@ -358,7 +358,8 @@ def run_native(args):
 
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 5), "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 5),
+        "ms_per_step_median": round(statistics.median(step_ms), 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 indexer / bf16 attention, fp32 accumulate",
         "data": "synthetic (seeded; dyadic FP8 indexer operands, N(0,1) bf16 latent/q/gate)",
         "config": {"workload": case.name, "batch_per_gpu": B, "context": Lctx, "indexer_heads": case.HI,
