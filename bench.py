@@ -533,6 +533,20 @@ def long_context_leg(args, flush, peaks, steps=100):
                 "unit": "GB/s", "frac": round(gbs / hbm, 4), "peak_spec": SPEC_HBM_GBS,
                 "frac_spec": round(gbs / SPEC_HBM_GBS, 4)}
 
+    def stages(lay, K=50):
+        """Stage split of the layer (separate steps, an event between stages)."""
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+        for e4 in ev:
+            for e in e4:
+                e.record()  # creates the handle
+        torch.cuda.synchronize()
+        for e4 in ev:
+            flush.zero_()
+            lay.forward_profiled(e4)
+        torch.cuda.synchronize()
+        return {k: round(sum(e4[i].elapsed_time(e4[i + 1]) for e4 in ev) / K * 1e3, 2)
+                for i, k in enumerate(["indexer", "topk", "attention"])}
+
     def device_ok(entry):
         err = _lib.device_error(reset=True)
         if err:
@@ -546,7 +560,8 @@ def long_context_leg(args, flush, peaks, steps=100):
         ms = ms_per_step(lay.forward)
         res["decode_1m"] = device_ok({"workload": c1.name, "us_per_step": round(ms * 1e3, 2),
                                       "tokens_per_s": round(c1.T / (ms * 1e-3), 1),
-                                      "roofline": hbm_roofline(decode_bytes(c1)[0], ms)})
+                                      "roofline": hbm_roofline(decode_bytes(c1)[0], ms),
+                                      "stages_us": stages(lay)})
         del lay, c1
     except Exception as e:  # recorded, not raised: the headline line must still print
         res["decode_1m"] = {"error": f"{type(e).__name__}: {e}"[:300]}
@@ -574,7 +589,7 @@ def long_context_leg(args, flush, peaks, steps=100):
         res["hybrid"] = device_ok({
             "workload": f"{hc.name} + 5 x swa_B{B}_H{H}_D{D}_W{sw.window}",
             "dsa_layer": {"us_per_step": round(dsa_ms * 1e3, 2),
-                          "roofline": hbm_roofline(decode_bytes(hc)[0], dsa_ms)},
+                          "roofline": hbm_roofline(decode_bytes(hc)[0], dsa_ms), "stages_us": stages(lay)},
             "swa_layer": {"us_per_step": round(swa_ms * 1e3, 2), "roofline": hbm_roofline(nbytes_swa, swa_ms)},
             "group_1_dsa_5_swa": {"us_per_step": round(group_ms * 1e3, 2),
                                   "tokens_per_s": round(B / (group_ms * 1e-3), 1)}})

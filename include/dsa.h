@@ -113,6 +113,27 @@ dsa_status dsa_topk(const float *scores, int64_t ld, const int32_t *row_len,
                     int32_t R, int32_t K, int32_t max_row_len, int32_t *idx,
                     void *ws, size_t ws_bytes, dsa_stream_t stream);
 
+/* ---- top-K given each row's coarse score histogram -------------------------
+ * Same result as dsa_topk, for rows whose scores the caller has already
+ * counted by their top 11 key bits (the indexer does this in the layer's
+ * decode path): hist[r*2048 + b] = number of positions s < row_len[r] whose
+ * key(scores[r*ld + s]) >> 21 == b, where key() maps an fp32 score to an
+ * order-preserving uint32 (bits flipped for negatives, sign bit set for
+ * non-negatives, -0.0 taken as +0.0).  One launch: every CTA lists the keys
+ * of its slice at or above the coarse bin of the K-th largest key, and the
+ * last CTA of each row selects among those.  A histogram that does not match
+ * the row only makes the call slower (the row is then selected in full).
+ *   hist   device uint32 [R, 2048]; read, then set to zero (so a caller that
+ *          counts into it again can reuse it)
+ *   ws     device scratch of dsa_topk_hist_workspace_bytes(R, max_row_len)
+ *          bytes, 256-byte aligned; contents need no initialisation.
+ *   scores 16-byte aligned, ld a multiple of 4.
+ * Supported: 1 <= K <= 4096. */
+size_t dsa_topk_hist_workspace_bytes(int32_t R, int32_t max_row_len);
+dsa_status dsa_topk_hist(const float *scores, int64_t ld, const int32_t *row_len,
+                         int32_t R, int32_t K, int32_t max_row_len, uint32_t *hist,
+                         int32_t *idx, void *ws, size_t ws_bytes, dsa_stream_t stream);
+
 /* ---- top-K with library-owned scratch ---------------------------------------
  * Not described by the source pages: an interface addition for callers that
  * cannot allocate device memory where the selection runs -- an engine whose
@@ -128,7 +149,8 @@ dsa_status dsa_topk(const float *scores, int64_t ld, const int32_t *row_len,
  *    before launching anything.
  *  - The first call on a device looks up the scratch array's device address
  *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before any stream capture begins.
+ *    before any stream capture begins.  A lookup that fails returns
+ *    DSA_ERR_CUDA and is tried again by the next call on that device.
  *  - Every call on a device shares the one array, which keeps the previous
  *    call's contents; each call clears what must start at zero.  Calls whose
  *    GPU work overlaps (different streams, no ordering between them) race on
@@ -190,8 +212,9 @@ typedef struct {
 } dsa_layer_args;
 
 /* Workspace: (decode, or T <= 64) a per-query histogram of the indexer scores, then the
- * fp32 scores [T, max_len] + top-K scratch (+ idx if idx_out is NULL) +
- * split-K attention partials.  Decode calls (and calls with T <= 64, such as
+ * fp32 scores [T, max_len] (+ idx if idx_out is NULL) + top-K scratch
+ * (dsa_topk_hist_workspace_bytes when the histogram is there, else
+ * dsa_topk_workspace_bytes) + split-K attention partials.  Decode calls (and calls with T <= 64, such as
  * several draft tokens per sequence) leave the histogram region zeroed and
  * take a faster top-K when they find it zeroed, so reusing one workspace
  * (zero-filled once, or simply reused after a first call) across such calls

@@ -64,6 +64,10 @@ lib.dsa_topk_workspace_bytes.restype = SZ
 lib.dsa_topk_workspace_bytes.argtypes = [I32, I32, I32]
 lib.dsa_topk.restype = ctypes.c_int
 lib.dsa_topk.argtypes = [P, I64, P, I32, I32, I32, P, P, SZ, P]
+lib.dsa_topk_hist_workspace_bytes.restype = SZ
+lib.dsa_topk_hist_workspace_bytes.argtypes = [I32, I32]
+lib.dsa_topk_hist.restype = ctypes.c_int
+lib.dsa_topk_hist.argtypes = [P, I64, P, I32, I32, I32, P, P, P, SZ, P]
 lib.dsa_topk_static.restype = ctypes.c_int
 lib.dsa_topk_static.argtypes = [P, I64, P, I32, I32, I32, P, P]
 lib.dsa_sparse_attn_workspace_bytes.restype = SZ
@@ -85,7 +89,7 @@ lib.dsa_swa_decode.restype = ctypes.c_int
 lib.dsa_swa_decode.argtypes = [P, P, P, P, I32, I32, I32, I32, F32, P, P]
 
 EXPORTS = ["dsa_abi_version", "dsa_status_string", "dsa_device_error", "dsa_indexer_scores",
-           "dsa_topk_workspace_bytes", "dsa_topk", "dsa_topk_static", "dsa_sparse_attn_workspace_bytes",
+           "dsa_topk_workspace_bytes", "dsa_topk", "dsa_topk_hist_workspace_bytes", "dsa_topk_hist", "dsa_topk_static", "dsa_sparse_attn_workspace_bytes",
            "dsa_sparse_attn",
            "dsa_layer_workspace_bytes", "dsa_layer_forward", "dsa_layer_forward_profiled",
            "dsa_layer_kernel_launches", "dsa_swa_decode", "dsa_append_kv"]
@@ -153,6 +157,21 @@ def topk(scores, row_len, K: int, max_row_len: int, idx=None, ws=None):
     _check("dsa_topk", lib.dsa_topk(
         _ptr(scores, torch.float32, "scores"), ld, _ptr(row_len, torch.int32, "row_len"), R, K, int(max_row_len),
         _ptr(idx, torch.int32, "idx"), _ptr(ws, torch.uint8, "ws", True), need if ws is None else ws.numel(),
+        _stream()))
+    return idx
+
+
+def topk_hist(scores, row_len, hist, K: int, max_row_len: int, idx=None, ws=None):
+    """hist uint32 (as torch.int32) [R, 2048]: counts of key(score) >> 21 per row; zeroed by the call."""
+    R, ld = scores.shape
+    if idx is None:
+        idx = torch.empty((R, K), dtype=torch.int32, device=scores.device)
+    need = int(lib.dsa_topk_hist_workspace_bytes(R, int(max_row_len)))
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=scores.device)
+    _check("dsa_topk_hist", lib.dsa_topk_hist(
+        _ptr(scores, torch.float32, "scores"), ld, _ptr(row_len, torch.int32, "row_len"), R, K, int(max_row_len),
+        _ptr(hist, torch.int32, "hist"), _ptr(idx, torch.int32, "idx"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
         _stream()))
     return idx
 

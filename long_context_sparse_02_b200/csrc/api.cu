@@ -56,9 +56,13 @@ bool ensure_smem(const void *fn, int bytes) {
     std::lock_guard<std::mutex> lk(g_smem_mu);
     for (auto &e : g_smem_done)
         if (e.first == fn && e.second == dev->device) return true;
-    // Raise the limit once to the device maximum, so later calls with a
-    // larger request need no new attribute call.
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dev->max_smem_optin) != cudaSuccess)
+    // Raise the limit once to the device maximum less the kernel's static
+    // shared memory, so later calls with a larger request need no new
+    // attribute call.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) return false;
+    const int limit = dev->max_smem_optin - (int)fa.sharedSizeBytes;
+    if (bytes > limit || cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, limit) != cudaSuccess)
         return false;
     g_smem_done.emplace_back(fn, dev->device);
     return true;
@@ -147,7 +151,10 @@ LayerWs carve_layer(const dsa_layer_args *a, void *ws) {
     } else {
         w.idx = a->idx_out;
     }
-    w.topk_bytes = topk_workspace_bytes(a->T, a->K, a->max_len);
+    // with the indexer's histogram the top-K lists candidates in a workspace of
+    // its own (its per-row tickets first); otherwise the plain top-K's
+    w.topk_bytes = hist_mode(a) ? topk_hist_workspace_bytes(a->T, a->max_len)
+                                : topk_workspace_bytes(a->T, a->K, a->max_len);
     w.topk_ws = w.topk_bytes ? p + off : nullptr;
     off += w.topk_bytes;
     w.attn_bytes = attn_workspace_bytes(a->T, a->H, a->K, a->Dv);
@@ -226,6 +233,28 @@ dsa_status dsa_topk_static(const float *scores, int64_t ld, const int32_t *row_l
     return launch_topk_static(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t dsa_topk_hist_workspace_bytes(int32_t R, int32_t max_row_len) {
+    if (R <= 0 || max_row_len <= 0) return 0;
+    return topk_hist_workspace_bytes(R, max_row_len);
+}
+
+dsa_status dsa_topk_hist(const float *scores, int64_t ld, const int32_t *row_len, int32_t R, int32_t K,
+                         int32_t max_row_len, uint32_t *hist, int32_t *idx, void *ws, size_t ws_bytes,
+                         dsa_stream_t stream) {
+    if (R < 0 || K < 1 || max_row_len < 1 || ld < max_row_len) return DSA_ERR_INVALID_ARG;
+    if (K > 4096) return DSA_ERR_UNSUPPORTED;
+    if (R == 0) return DSA_OK;
+    if (!scores || !row_len || !hist || !idx || !aligned16(scores) || (ld & 3)) return DSA_ERR_INVALID_ARG;
+    const size_t need = topk_hist_workspace_bytes(R, max_row_len);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return DSA_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // the counters at the head of the workspace start at zero
+    if (cudaMemsetAsync(ws, 0, (size_t)topk_hist_zero_words(R) * 4, st) != cudaSuccess) return DSA_ERR_CUDA;
+    TopkArgs a{scores, ld, row_len, ROWLEN_ARRAY, R, K, max_row_len, idx, ws, ws_bytes};
+    a.hist = hist;
+    return launch_topk_hist(a, st);
+}
+
 size_t dsa_sparse_attn_workspace_bytes(int32_t T, int32_t H, int32_t K, int32_t Dv) {
     if (T <= 0 || H <= 0 || K < 64) return 0;
     return attn_workspace_bytes(T, H, K, Dv);
@@ -282,7 +311,9 @@ dsa_status layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes, dsa
     const PagedDev pg = paged_dev(&a->pg);
     const int64_t ld = (int64_t)ld_of(a->max_len);
     IndexerArgs ia{a->q_idx, a->w, a->k_idx_cache, pg, decode ? nullptr : a->q_seq, decode ? nullptr : a->q_pos,
-                   a->T, a->HI, a->DI, a->max_len, lw.scores, ld, hist_mode(a) ? lw.score_hist : nullptr};
+                   a->T, a->HI, a->DI, a->max_len, lw.scores, ld, hist_mode(a) ? lw.score_hist : nullptr,
+                   hist_mode(a) ? static_cast<uint32_t *>(lw.topk_ws) : nullptr,
+                   hist_mode(a) ? topk_hist_zero_words(a->T) : 0};
     if (!mark(0)) return DSA_ERR_CUDA;
     dsa_status s = launch_indexer(ia, st);
     if (s != DSA_OK) return s;
@@ -291,8 +322,17 @@ dsa_status layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes, dsa
                 decode ? (int32_t)ROWLEN_SEQ_LENS : (int32_t)ROWLEN_QPOS_PLUS_1,
                 a->T, a->K, a->max_len, lw.idx, lw.topk_ws, lw.topk_bytes};
     ta.pdl = true;
-    if (hist_mode(a)) ta.hist = lw.score_hist;
-    s = launch_topk(ta, st);
+    if (hist_mode(a)) {
+        ta.hist = lw.score_hist;
+        if (topk_prefers_cluster(a->T, a->max_len)) {
+            ta.ws = nullptr, ta.ws_bytes = 0;  // the cluster kernel needs none
+            s = launch_topk(ta, st);
+        } else {
+            s = launch_topk_hist(ta, st);
+        }
+    } else {
+        s = launch_topk(ta, st);
+    }
     if (s != DSA_OK) return s;
     if (!mark(2)) return DSA_ERR_CUDA;
     AttnArgs aa{a->q, a->kv_cache, pg, decode ? nullptr : a->q_seq, lw.idx, a->K, a->gate, a->sm_scale, a->T, a->H,
@@ -317,7 +357,7 @@ dsa_status dsa_layer_forward_profiled(const dsa_layer_args *a, void *ws, size_t 
 
 int32_t dsa_layer_kernel_launches(const dsa_layer_args *a) {
     if (!a || a->T <= 0 || a->max_len < 1) return 0;
-    return 1 + topk_kernel_launches(a->T, a->max_len) + attn_kernel_launches(a->T, a->K, a->Dv);
+    return 1 + (hist_mode(a) ? 1 : topk_kernel_launches(a->T, a->max_len)) + attn_kernel_launches(a->T, a->K, a->Dv);
 }
 
 dsa_status dsa_append_kv(const uint16_t *k_new, float k_scale, const uint16_t *latent_new, const int32_t *tok_seq,

@@ -51,9 +51,13 @@ struct IndexerArgs {
     int32_t T, HI, DI, max_len;
     float *scores;
     int64_t ld;
-    // optional (decode convention only): per-query histogram [T][SCORE_HIST_BINS]
+    // optional (few-query kernels only): per-query histogram [T][SCORE_HIST_BINS]
     // of score_key(score) >> SCORE_HIST_SHIFT, added to (it must hold zeros)
     uint32_t *hist;
+    // optional: words the kernel sets to zero before it ends (the counters
+    // of the top-K that follows it)
+    uint32_t *zero;
+    int64_t nzero;
 };
 constexpr int SCORE_HIST_BINS = 2048;
 constexpr int SCORE_HIST_SHIFT = 21;
@@ -81,8 +85,26 @@ struct TopkArgs {
 };
 size_t topk_workspace_bytes(int32_t R, int32_t K, int32_t max_row_len);
 int topk_kernel_launches(int32_t R, int32_t max_row_len);
+// Few rows that each fit one large thread-block cluster (10 or 16 CTAs, all
+// clusters resident at once): the cluster kernel, which also reads the
+// indexer's histogram, selects faster than the single-launch list-and-ticket
+// kernel; longer rows and many rows go to the latter.
+bool topk_prefers_cluster(int32_t R, int32_t max_row_len);
 dsa_status launch_topk(const TopkArgs &a, cudaStream_t st);
 dsa_status launch_topk_static(const TopkArgs &a, cudaStream_t st);
+// Top-K from the indexer's per-row histogram (a.hist set): one launch, every
+// CTA lists its slice's keys at or above the threshold's coarse bin, the
+// last CTA of each row (atomic ticket) selects.  a.ws is its workspace, whose
+// first topk_hist_zero_words(R) words (fine counts and tickets) must be zero
+// at launch: the indexer zeroes them (IndexerArgs::zero), and the top-K
+// leaves them zeroed.
+struct HistTopkPlan {
+    int S, slice;  // CTAs per row, keys per CTA
+};
+HistTopkPlan topk_hist_plan(int32_t R, int32_t max_row_len);
+size_t topk_hist_workspace_bytes(int32_t R, int32_t max_row_len);
+int64_t topk_hist_zero_words(int32_t R);
+dsa_status launch_topk_hist(const TopkArgs &a, cudaStream_t st);
 
 // ---- gated sparse attention ----------------------------------------------------
 struct AttnArgs {

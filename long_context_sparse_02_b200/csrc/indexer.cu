@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(DecCfg<DI, NH>::THREADS, DecCfg<DI, NH>::CTAS_
     }
     if (p.hist)
         for (int i = threadIdx.x; i < C::EPI_GROUPS * C::HIST_WORDS; i += blockDim.x) hist_sm[i] = 0;
+    clear_words(p);
 
     if (threadIdx.x == 32) {
         for (int s = 0; s < C::STAGES; ++s) {
@@ -763,7 +764,8 @@ dsa_status launch_indexer(const IndexerArgs &a, cudaStream_t st) {
     if (a.T == 0) return DSA_OK;
     if (indexer_group_eligible(a)) return launch_indexer_group(a, st);
     IdxParams p{a.w, a.q_seq, a.q_pos, a.pg, a.T, a.HI, a.max_len, a.scores, a.ld, dev->err,
-                (a.q_seq == nullptr || a.T <= 64) ? a.hist : nullptr};  // the few-query kernel counts
+                (a.q_seq == nullptr || a.T <= 64) ? a.hist : nullptr,  // the few-query kernel counts
+                a.zero, a.nzero};
     const CUtensorMapSwizzle swz = a.DI == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUtensorMap km, qm;
     if (!make_tmap_2d(&km, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.DI, (uint64_t)a.pg.num_pages * 64, a.DI,

@@ -73,7 +73,16 @@ struct IdxParams {
     int64_t ld;
     uint32_t *err;
     uint32_t *hist;  // [T][SCORE_HIST_BINS] or NULL (few-query kernels only)
+    uint32_t *zero;  // nzero words the grid sets to zero (or NULL)
+    int64_t nzero;
 };
+
+// The grid clears the words the next kernel expects at zero, each CTA a share.
+__device__ __forceinline__ void clear_words(const IdxParams &p) {
+    if (p.zero)
+        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.nzero; i += (int64_t)gridDim.x * blockDim.x)
+            p.zero[i] = 0;
+}
 
 // Index t with tstart[t] <= g < tstart[t+1] (tstart non-decreasing, g < tstart[T]).
 __device__ __forceinline__ int locate(const int32_t *tstart, int T, int64_t g) {

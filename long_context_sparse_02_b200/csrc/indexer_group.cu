@@ -85,6 +85,7 @@ __global__ void __launch_bounds__(GrpCfg<NH>::THREADS, 1)
         for (int i = threadIdx.x; i < C::EPI_GROUPS * GQ * C::HIST_WORDS; i += blockDim.x) hist_sm[i] = 0;
     for (int i = threadIdx.x; i < T * NH; i += blockDim.x)
         wsm[i] = (i % NH) < p.HI ? p.w[(int64_t)(i / NH) * p.HI + (i % NH)] : 0.f;
+    clear_words(p);
     if (threadIdx.x == 32) {
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
@@ -368,7 +369,7 @@ dsa_status launch_indexer_group(const IndexerArgs &a, cudaStream_t st) {
     const DeviceInfo *dev = current_device();
     if (!dev) return DSA_ERR_CUDA;
     if (!indexer_group_eligible(a)) return DSA_ERR_UNSUPPORTED;
-    IdxParams p{a.w, a.q_seq, a.q_pos, a.pg, a.T, a.HI, a.max_len, a.scores, a.ld, dev->err, a.hist};
+    IdxParams p{a.w, a.q_seq, a.q_pos, a.pg, a.T, a.HI, a.max_len, a.scores, a.ld, dev->err, a.hist, a.zero, a.nzero};
     CUtensorMap km, qm;
     if (!make_tmap_2d(&km, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.DI, (uint64_t)a.pg.num_pages * 64, a.DI,
                       a.DI, 64, CU_TENSOR_MAP_SWIZZLE_128B))

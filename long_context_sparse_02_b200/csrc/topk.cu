@@ -1308,6 +1308,11 @@ size_t topk_workspace_bytes(int32_t R, int32_t K, int32_t max_row_len) {
     return align_up(multi_zero_bytes(R) + (size_t)R * nch * 2 * 4, 256);
 }
 
+bool topk_prefers_cluster(int32_t R, int32_t max_row_len) {
+    const DeviceInfo *dev = current_device();
+    return dev && cluster_plan(R, max_row_len, dev).cl >= 10;
+}
+
 int topk_kernel_launches(int32_t R, int32_t max_row_len) {
     const DeviceInfo *dev = current_device();
     return (dev && cluster_plan(R, max_row_len, dev).cl > 0) ? 1 : 5;
@@ -1355,9 +1360,8 @@ static_assert(STATIC_SCRATCH_BYTES == DSA_TOPK_STATIC_SCRATCH_BYTES, "header sta
 static __device__ __align__(256) uint8_t g_topk_static_scratch[STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDev = 64;
-std::once_flag g_static_once[kMaxDev];
-void *g_static_ptr[kMaxDev];
-cudaError_t g_static_rc[kMaxDev];
+std::mutex g_static_mu;
+void *g_static_ptr[kMaxDev];  // set once a lookup on that device has succeeded
 }  // namespace
 
 dsa_status launch_topk_static(const TopkArgs &a, cudaStream_t st) {
@@ -1366,16 +1370,25 @@ dsa_status launch_topk_static(const TopkArgs &a, cudaStream_t st) {
     if (a.R > STATIC_MAX_ROWS || a.max_row_len > STATIC_MAX_ROW_LEN) return DSA_ERR_UNSUPPORTED;
     if (a.R == 0) return DSA_OK;
     const int d = dev->device;
-    std::call_once(g_static_once[d], [d] {
-        void *p = nullptr;
-        g_static_rc[d] = cudaGetSymbolAddress(&p, g_topk_static_scratch);
-        g_static_ptr[d] = p;
-    });
-    if (g_static_rc[d] != cudaSuccess || !g_static_ptr[d]) return DSA_ERR_CUDA;
-    MultiWs m = carve_multi(g_static_ptr[d], a.R, a.max_row_len);
+    void *scratch = nullptr;
+    {
+        // Only a successful lookup is kept: a call that failed (made during a
+        // stream capture, say) returns DSA_ERR_CUDA and the next call tries again.
+        std::lock_guard<std::mutex> lk(g_static_mu);
+        if (!g_static_ptr[d]) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_topk_static_scratch) != cudaSuccess || !p) {
+                cudaGetLastError();
+                return DSA_ERR_CUDA;
+            }
+            g_static_ptr[d] = p;
+        }
+        scratch = g_static_ptr[d];
+    }
+    MultiWs m = carve_multi(scratch, a.R, a.max_row_len);
     // Histograms, tickets and row state must start at zero; the array keeps
     // whatever the previous call left.
-    if (cudaMemsetAsync(g_static_ptr[d], 0, multi_zero_bytes(a.R), st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaMemsetAsync(scratch, 0, multi_zero_bytes(a.R), st) != cudaSuccess) return DSA_ERR_CUDA;
     dim3 grid(m.nchunks, a.R);
     for (int ps = 0; ps < 3; ++ps) topk_pass_kernel<<<grid, MULTI_THREADS, 0, st>>>(a, m, ps, dev->err);
     topk_count_kernel<<<grid, MULTI_THREADS, 0, st>>>(a, m);

@@ -107,13 +107,21 @@ def test_host_side_argument_errors(lib):
     # zero-sized calls are no-ops
     assert L.dsa_append_kv(None, 1.0, None, None, None, ctypes.byref(ok_pg), 0, 128, 0, None, None, None) == 0
     assert L.dsa_topk(P(16), 10, P(16), 0, 8, 10, P(16), None, 0, None) == 0
+    # histogram-fed top-K: bad K, ld below the row length, misaligned scores, no histogram, no workspace
+    assert L.dsa_topk_hist(P(16), 100, P(16), 4, 5000, 100, P(16), P(16), None, 0, None) == 2
+    assert L.dsa_topk_hist(P(16), 50, P(16), 4, 8, 100, P(16), P(16), None, 0, None) == 1
+    assert L.dsa_topk_hist(P(20), 100, P(16), 4, 8, 100, P(16), P(16), None, 0, None) == 1
+    assert L.dsa_topk_hist(P(16), 100, P(16), 4, 8, 100, None, P(16), None, 0, None) == 1
+    assert L.dsa_topk_hist(P(16), 100, P(16), 4, 8, 100, P(16), P(16), None, 0, None) == 3
+    assert L.dsa_topk_hist(P(16), 10, P(16), 0, 8, 10, P(16), P(16), None, 0, None) == 0
 
 
 def test_layer_workspace_follows_the_documented_layout(lib):
     """dsa_layer_workspace_bytes (host only) adds up the regions dsa.h lists:
     the per-query score histogram (2048 bins of 4 bytes, in decode and for
     T <= 64), the fp32 score rows (ld = max_len rounded up to 4), the idx rows
-    when idx_out is NULL, then the top-K and attention scratch; each of the
+    when idx_out is NULL, then the top-K scratch (the histogram-fed top-K's
+    whenever the histogram is there) and the attention scratch; each of the
     first three regions 256-byte aligned.  runtime.LayerOnDevice.scores reads
     the score rows behind that histogram region."""
     from long_context_sparse_02_b200._lib import LayerArgs
@@ -135,8 +143,10 @@ def test_layer_workspace_follows_the_documented_layout(lib):
                 assert ws(mode, T, max_len) - base == up(T * 2048 * 4)
                 hist = up(T * 2048 * 4) if (mode == 1 or T <= 64) else 0
                 rows = up(T * ((max_len + 3) // 4 * 4) * 4)
-                scratch = L.dsa_topk_workspace_bytes(T, 2048, max_len) + L.dsa_sparse_attn_workspace_bytes(T, 128,
-                                                                                                          2048, 512)
+                topk = L.dsa_topk_hist_workspace_bytes(T, max_len) if hist else \
+                    L.dsa_topk_workspace_bytes(T, 2048, max_len)
+                scratch = topk + L.dsa_sparse_attn_workspace_bytes(T, 128, 2048, 512)
                 assert base == hist + rows + scratch, (T, mode, max_len)
-    assert ws(1, 65, 1000) - ws(0, 65, 1000) == up(65 * 2048 * 4)
+    assert ws(1, 65, 1000) - ws(0, 65, 1000) == up(65 * 2048 * 4) + L.dsa_topk_hist_workspace_bytes(65, 1000) - \
+        L.dsa_topk_workspace_bytes(65, 2048, 1000)
     assert ws(0, 0, 10) == 0 and ws(0, 4, 0) == 0 and ws(0, 4, 10, K=0) == 0

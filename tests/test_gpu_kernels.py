@@ -155,6 +155,47 @@ def test_topk_bit_exact(L, orc, R, n, K, kind):
     no_device_error(L)
 
 
+def coarse_hist(sc, rl):
+    """Counts of each row's order-preserving score keys by their top 11 bits
+    (the caller-side input of dsa_topk_hist; -0.0 counts as +0.0)."""
+    u = sc.astype(np.float32).view(np.uint32).copy()
+    u[u == 0x80000000] = 0
+    key = np.where(u & 0x80000000, ~u, u | 0x80000000).astype(np.uint32)
+    h = np.zeros((sc.shape[0], 2048), np.int64)
+    for r in range(sc.shape[0]):
+        h[r] = np.bincount(key[r, :rl[r]] >> 21, minlength=2048)
+    return h.astype(np.uint32).view(np.int32)
+
+
+@pytest.mark.parametrize("R,n,K,kind", TOPK_CASES, ids=[f"{c[0]}x{c[1]}_K{c[2]}_{c[3]}" for c in TOPK_CASES])
+def test_topk_hist_bit_exact(L, orc, R, n, K, kind):
+    """The histogram-fed top-K (one launch, last-CTA select) on the same rows,
+    twice on one workspace; a garbage histogram takes the whole-row select."""
+    sc = synth.score_rows(11, R, n, kind)
+    ld = (n + 3) // 4 * 4
+    scp = np.zeros((R, ld), np.float32)
+    scp[:, :n] = sc
+    rng = np.random.default_rng(12)
+    rl = rng.integers(0, n + 1, size=R).astype(np.int32)
+    rl[0] = n
+    if R > 2:
+        rl[1], rl[2] = min(K, n), min(K + 1, n)
+    ref = orc.topk(sc, rl, K)
+    hist = dev(coarse_hist(sc, rl))
+    ws = torch.full((L.lib.dsa_topk_hist_workspace_bytes(R, n),), 0x5A, dtype=torch.uint8, device="cuda")
+    for rep in range(3):
+        if rep == 2:  # counts that do not describe the rows
+            hist = torch.randint(0, 64, (R, 2048), dtype=torch.int32, device="cuda")
+        elif rep == 1:
+            assert int(hist.abs().sum()) == 0  # the first call cleared the counts
+            hist = dev(coarse_hist(sc, rl))
+        idx = L.topk_hist(dev(scp), dev(rl), hist, K, n, ws=ws)
+        got = idx.cpu().numpy()
+        for r in range(R):
+            assert np.array_equal(got[r], ref[r]), (rep, r, rl[r])
+    no_device_error(L)
+
+
 # ------------------------------------------------------------------ attention
 
 @pytest.mark.parametrize("Dqk,Dv,H,K,seq_lens,T,pad", [
