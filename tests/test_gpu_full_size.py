@@ -13,6 +13,9 @@ The same calls and launch configurations the benchmark times:
   dsa_indexer_scores and dsa_topk over all 32768 rows -- scores and indices of
   sampled rows (the first, last and tile-boundary rows plus seeded random ones)
   compared bit for bit with the oracle, which computes those rows alone;
+* the whole prefill layer at T = 32768 (16x128 indexer, 128 heads) through
+  dsa_layer_forward -- indices and outputs of a fixed row set (rows 0-63,
+  2040-2056, the last 64, 256 seeded random rows);
 * the hybrid serving step: 64 decode sequences with lengths uniform in
   [4096, 65536] through one DSA layer (16x128 indexer) and one sliding-window
   layer (64 heads x 128, window 128) -- every element compared.
@@ -126,6 +129,35 @@ def test_prefill_T32768_indexer_and_topk_sampled_rows(L, orc):
     assert np.array_equal(idx[torch.from_numpy(rows).cuda()].cpu().numpy(), ref_idx)
     del scores, idx
     torch.cuda.empty_cache()
+
+
+def test_prefill_T32768_layer_sampled_rows(L, orc):
+    """The whole prefill layer at its full size (one sequence of 32768 causal
+    queries, 16x128 indexer, K = 2048, 128 heads over the 576-wide latent,
+    gated) through dsa_layer_forward, checked on a fixed row set: rows 0-63,
+    2040-2056, the last 64 and 256 seeded random rows -- indices bit for bit
+    against the oracle's scores and top-K of those rows, outputs within the
+    bf16 tolerance against the oracle's attention over them."""
+    from long_context_sparse_02_b200.runtime import LayerOnDevice
+    T = 32768
+    c = synth.prefill_case(7, T)
+    lay = LayerOnDevice(c, decode=False)
+    lay.forward()
+    torch.cuda.synchronize()
+    assert L.device_error(reset=True) == 0
+    rows = np.unique(np.r_[np.arange(64), np.arange(2040, 2057), np.arange(T - 64, T),
+                           np.random.default_rng(17).integers(0, T, 256)]).astype(np.int64)
+    sel = torch.from_numpy(rows).cuda()
+    got_idx = lay.idx[sel].cpu().numpy()
+    got_out = lay.out[sel].float().cpu().numpy().astype(np.float64)
+    del lay
+    torch.cuda.empty_cache()
+    pg = orc.Paged(c.seq_lens, c.block_table, 64, c.num_pages)
+    sc = orc.indexer_scores(c.q_idx[rows], c.w[rows], c.k_cache, pg, c.q_seq[rows], c.q_pos[rows], ld=T)
+    ref_idx = orc.topk(sc, c.q_pos[rows] + 1, c.K)
+    assert np.array_equal(got_idx, ref_idx), "indices differ"
+    ref_out = orc.sparse_attn(c.q[rows], c.kv_cache, pg, c.q_seq[rows], ref_idx, c.gate[rows], c.sm_scale, c.Dv)
+    assert_attn_close(got_out, ref_out)
 
 
 def test_hybrid_B64_dsa_and_swa_full(L, orc):
