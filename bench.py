@@ -76,6 +76,9 @@ def parse_args(argv=None):
                     help="time only the prefill indexer at T queries (small cases for profiling)")
     ap.add_argument("--append-only", action="store_true",
                     help="time only the append step (dsa_append_kv), for profiling")
+    ap.add_argument("--workload", choices=["decode", "cp_decode_1m"], default="decode",
+                    help="cp_decode_1m: one 1,048,576-token sequence's history split over the N ranks "
+                         "(context-parallel decode, two NCCL all-gathers per step)")
     return ap.parse_args(argv)
 
 
@@ -957,10 +960,71 @@ def run_reference(args):
     print(json.dumps(res), flush=True)
 
 
+def run_cp(args):
+    """Context-parallel decode of one 1,048,576-token sequence over the N
+    ranks: every rank holds the caches (it reads only its own pages), runs
+    its local indexer and top-K, all-gathers the candidates, attends over the
+    kept rows it holds, all-gathers (output, log-sum-exp) and merges.  The
+    step time is the max over ranks of the CUDA-event time of K steps
+    (the exchanges included); one token per step."""
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+    from long_context_sparse_02_b200 import build, synth
+    build.build()
+    from long_context_sparse_02_b200 import _lib, cp
+    from long_context_sparse_02_b200.runtime import to_dev
+    c = synth.decode_1m(args.seed)
+    k_cache, kv_cache = to_dev(c.k_cache), to_dev(c.kv_cache)
+    q_idx, w, q, gate = to_dev(c.q_idx), to_dev(c.w), to_dev(c.q), to_dev(c.gate)
+    rk = cp.CpRank(rank, world, c.seq_lens, c.block_table, c.num_pages, k_cache, kv_cache, c.K, c.Dv, c.sm_scale)
+    if world > 1:
+        ag = cp.torch_all_gather()
+        step = lambda: cp.decode_step(rk, q_idx, w, q, gate, ag)  # noqa: E731
+    else:
+        step = lambda: cp.emulate([rk], q_idx, w, q, gate)  # noqa: E731
+    flush = L2Flush()
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    total = 0.0
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        torch.cuda.synchronize()
+        total += e0.elapsed_time(e1)
+    if world > 1:
+        torch.distributed.barrier()
+    max_ms, _ = aggregate(total, args.steps, world)
+    err = _lib.device_error(reset=True)
+    res = {"metric": "context-parallel decode tokens/s, one 1,048,576-token sequence", "value":
+           round(args.steps / (max_ms / 1e3), 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 5), "higher_is_better": True,
+           "scaling": "strong", "vs_baseline": None, "dtype": "e4m3 indexer / bf16 attention, fp32 accumulate",
+           "data": "synthetic (seeded)", "config": {"workload": c.name, "parallelism": f"cp{world}",
+                                                    "l2": "flushed between timed steps"},
+           "device_error": err}
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
 if __name__ == "__main__":
     a = parse_args()
     if a.impl == "reference":
         run_reference(a)
+    elif a.workload == "cp_decode_1m":
+        run_cp(a)
     elif a.prefill_only:
         import torch
         from long_context_sparse_02_b200 import build

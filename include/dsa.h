@@ -268,6 +268,49 @@ dsa_status dsa_append_kv(const uint16_t *k_new, float k_scale, const uint16_t *l
                          int32_t n, int32_t DI, int32_t Dqk, uint8_t *k_idx_cache,
                          uint16_t *kv_cache, dsa_stream_t stream);
 
+/* ---- context-parallel decode: one long sequence over G GPUs -----------------------
+ * "Fine-Grained Sparse Attention in Ultra-Large Parameter Models", §1
+ * (1,048,576-token context); "Open-Weight Deployment of an Ultra-Large Sparse
+ * Model", §3 (multi-card deployment).  The pages describe no split; this one
+ * deals every sequence's pages out in G contiguous runs of whole pages, rank r
+ * holding positions [lo[b], hi[b]) of sequence b.  Per rank, per decode step:
+ *   1. dsa_indexer_scores and dsa_topk over the rank's own pages (a paged view
+ *      whose seq_lens are hi - lo and whose block table starts at page lo/64),
+ *      giving local scores and local indices;
+ *   2. dsa_cp_candidates: (score, global position) of each kept local index;
+ *   3. the caller all-gathers the G ranks' [B, K] candidate blocks (NCCL) into
+ *      [G, B, K] arrays, rank order;
+ *   4. dsa_cp_select: the K best of the G*K candidates of each sequence under
+ *      the top-K's order -- exactly the one-GPU selection, since a position
+ *      among the K best of the history is among the K best of its own range --
+ *      as global positions (ascending, -1 padded) and as this rank's local
+ *      indices (position - lo, -1 where another rank holds the row);
+ *   5. dsa_sparse_attn over the local indices with lse: the rank's gated
+ *      partial output and log-sum-exp (-inf where it holds no kept row);
+ *   6. the caller all-gathers o [G, B, H, Dv] and lse [G, B, H];
+ *   7. dsa_cp_lse_merge: out = sum_r w_r o_r / sum_r w_r, w_r = exp(lse_r -
+ *      max lse), over the ranks that hold a kept row.  (The gate is the same
+ *      factor in every rank's term.)
+ * All pointers are device memory; all calls are stream-ordered. */
+/*   scores [B, ld] local scores; idx_local [B, K] dsa_topk output; lo device int32 [B];
+ *   cand_score fp32 [B, K], cand_pos int32 [B, K] (padding: -inf, -1). */
+dsa_status dsa_cp_candidates(const float *scores, int64_t ld, const int32_t *idx_local,
+                             int32_t B, int32_t K, const int32_t *lo, float *cand_score,
+                             int32_t *cand_pos, dsa_stream_t stream);
+/*   cand_score, cand_pos [G, B, K] (every rank's candidates, rank order); lo, hi
+ *   device int32 [B] (this rank's range); idx_global, idx_local int32 [B, K];
+ *   ws of dsa_cp_select_workspace_bytes(G, B, K) bytes, 256-byte aligned.
+ *   Supported: K <= 4096, G * K <= 2^24. */
+size_t dsa_cp_select_workspace_bytes(int32_t G, int32_t B, int32_t K);
+dsa_status dsa_cp_select(const float *cand_score, const int32_t *cand_pos, int32_t G,
+                         int32_t B, int32_t K, const int32_t *lo, const int32_t *hi,
+                         int32_t *idx_global, int32_t *idx_local, void *ws, size_t ws_bytes,
+                         dsa_stream_t stream);
+/*   o bf16 [G, B, H, Dv], lse fp32 [G, B, H]; out bf16 [B, H, Dv].  Dv % 8 == 0,
+ *   o and out 16-byte aligned. */
+dsa_status dsa_cp_lse_merge(const uint16_t *o, const float *lse, int32_t G, int32_t B,
+                            int32_t H, int32_t Dv, uint16_t *out, dsa_stream_t stream);
+
 /* ---- housekeeping ---------------------------------------------------------------- */
 const char *dsa_status_string(dsa_status s);
 int32_t dsa_abi_version(void);

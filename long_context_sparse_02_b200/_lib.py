@@ -85,6 +85,14 @@ lib.dsa_layer_kernel_launches.restype = I32
 lib.dsa_append_kv.restype = ctypes.c_int
 lib.dsa_append_kv.argtypes = [P, F32, P, P, P, ctypes.POINTER(Paged), I32, I32, I32, P, P, P]
 lib.dsa_layer_kernel_launches.argtypes = [ctypes.POINTER(LayerArgs)]
+lib.dsa_cp_candidates.restype = ctypes.c_int
+lib.dsa_cp_candidates.argtypes = [P, I64, P, I32, I32, P, P, P, P]
+lib.dsa_cp_select_workspace_bytes.restype = SZ
+lib.dsa_cp_select_workspace_bytes.argtypes = [I32, I32, I32]
+lib.dsa_cp_select.restype = ctypes.c_int
+lib.dsa_cp_select.argtypes = [P, P, I32, I32, I32, P, P, P, P, P, SZ, P]
+lib.dsa_cp_lse_merge.restype = ctypes.c_int
+lib.dsa_cp_lse_merge.argtypes = [P, P, I32, I32, I32, I32, P, P]
 lib.dsa_swa_decode.restype = ctypes.c_int
 lib.dsa_swa_decode.argtypes = [P, P, P, P, I32, I32, I32, I32, F32, P, P]
 
@@ -92,7 +100,8 @@ EXPORTS = ["dsa_abi_version", "dsa_status_string", "dsa_device_error", "dsa_inde
            "dsa_topk_workspace_bytes", "dsa_topk", "dsa_topk_hist_workspace_bytes", "dsa_topk_hist", "dsa_topk_static", "dsa_sparse_attn_workspace_bytes",
            "dsa_sparse_attn",
            "dsa_layer_workspace_bytes", "dsa_layer_forward", "dsa_layer_forward_profiled",
-           "dsa_layer_kernel_launches", "dsa_swa_decode", "dsa_append_kv"]
+           "dsa_layer_kernel_launches", "dsa_swa_decode", "dsa_append_kv", "dsa_cp_candidates",
+           "dsa_cp_select_workspace_bytes", "dsa_cp_select", "dsa_cp_lse_merge"]
 
 
 def _check(fn: str, status: int):
@@ -254,3 +263,46 @@ def append_kv(k_new, k_scale: float, latent_new, tok_seq, tok_pos, pg: Paged, k_
         _ptr(k_new, torch.bfloat16, "k_new"), float(k_scale), _ptr(latent_new, torch.bfloat16, "latent_new", True),
         _ptr(tok_seq, torch.int32, "tok_seq"), _ptr(tok_pos, torch.int32, "tok_pos"), ctypes.byref(pg), n, DI, Dqk,
         _ptr(k_cache, torch.uint8, "k_cache"), _ptr(kv_cache, torch.bfloat16, "kv_cache", True), _stream()))
+
+
+def cp_candidates(scores, idx_local, lo, cand_score=None, cand_pos=None):
+    """(score, global position) of each locally kept index; scores fp32 [B, ld], idx_local int32 [B, K]."""
+    B, K = idx_local.shape
+    if cand_score is None:
+        cand_score = torch.empty((B, K), dtype=torch.float32, device=scores.device)
+    if cand_pos is None:
+        cand_pos = torch.empty((B, K), dtype=torch.int32, device=scores.device)
+    _check("dsa_cp_candidates", lib.dsa_cp_candidates(
+        _ptr(scores, torch.float32, "scores"), int(scores.shape[1]), _ptr(idx_local, torch.int32, "idx_local"), B, K,
+        _ptr(lo, torch.int32, "lo"), _ptr(cand_score, torch.float32, "cand_score"),
+        _ptr(cand_pos, torch.int32, "cand_pos"), _stream()))
+    return cand_score, cand_pos
+
+
+def cp_select(cand_score, cand_pos, lo, hi, idx_global=None, idx_local=None, ws=None):
+    """cand_score fp32 / cand_pos int32 [G, B, K] (every rank's candidates) -> (idx_global, idx_local) [B, K]."""
+    G, B, K = cand_score.shape
+    dev = cand_score.device
+    if idx_global is None:
+        idx_global = torch.empty((B, K), dtype=torch.int32, device=dev)
+    if idx_local is None:
+        idx_local = torch.empty((B, K), dtype=torch.int32, device=dev)
+    need = int(lib.dsa_cp_select_workspace_bytes(G, B, K))
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check("dsa_cp_select", lib.dsa_cp_select(
+        _ptr(cand_score, torch.float32, "cand_score"), _ptr(cand_pos, torch.int32, "cand_pos"), G, B, K,
+        _ptr(lo, torch.int32, "lo"), _ptr(hi, torch.int32, "hi"), _ptr(idx_global, torch.int32, "idx_global"),
+        _ptr(idx_local, torch.int32, "idx_local"), _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream()))
+    return idx_global, idx_local
+
+
+def cp_lse_merge(o, lse, out=None):
+    """o bf16 [G, B, H, Dv], lse fp32 [G, B, H] -> out bf16 [B, H, Dv]."""
+    G, B, H, Dv = o.shape
+    if out is None:
+        out = torch.empty((B, H, Dv), dtype=torch.bfloat16, device=o.device)
+    _check("dsa_cp_lse_merge", lib.dsa_cp_lse_merge(
+        _ptr(o, torch.bfloat16, "o"), _ptr(lse, torch.float32, "lse"), G, B, H, Dv, _ptr(out, torch.bfloat16, "out"),
+        _stream()))
+    return out

@@ -374,6 +374,39 @@ dsa_status dsa_append_kv(const uint16_t *k_new, float k_scale, const uint16_t *l
     return launch_append(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+dsa_status dsa_cp_candidates(const float *scores, int64_t ld, const int32_t *idx_local, int32_t B, int32_t K,
+                             const int32_t *lo, float *cand_score, int32_t *cand_pos, dsa_stream_t stream) {
+    if (B < 0 || K < 1 || ld < 1) return DSA_ERR_INVALID_ARG;
+    if (B == 0) return DSA_OK;
+    if (!scores || !idx_local || !lo || !cand_score || !cand_pos) return DSA_ERR_INVALID_ARG;
+    return launch_cp_candidates(scores, ld, idx_local, B, K, lo, cand_score, cand_pos,
+                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_cp_select_workspace_bytes(int32_t G, int32_t B, int32_t K) {
+    if (G < 1 || B < 1 || K < 1 || (int64_t)G * K > (1 << 24)) return 0;
+    return cp_select_workspace_bytes(G, B, K);
+}
+
+dsa_status dsa_cp_select(const float *cand_score, const int32_t *cand_pos, int32_t G, int32_t B, int32_t K,
+                         const int32_t *lo, const int32_t *hi, int32_t *idx_global, int32_t *idx_local, void *ws,
+                         size_t ws_bytes, dsa_stream_t stream) {
+    if (G < 1 || B < 0 || K < 1 || (int64_t)G * K > (1 << 24)) return DSA_ERR_INVALID_ARG;
+    if (K > 4096) return DSA_ERR_UNSUPPORTED;
+    if (B == 0) return DSA_OK;
+    if (!cand_score || !cand_pos || !lo || !hi || !idx_global || !idx_local) return DSA_ERR_INVALID_ARG;
+    return launch_cp_select(cand_score, cand_pos, G, B, K, lo, hi, idx_global, idx_local, ws, ws_bytes,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_cp_lse_merge(const uint16_t *o, const float *lse, int32_t G, int32_t B, int32_t H, int32_t Dv,
+                            uint16_t *out, dsa_stream_t stream) {
+    if (G < 1 || B < 0 || H < 1 || Dv < 8 || Dv % 8) return DSA_ERR_INVALID_ARG;
+    if (B == 0) return DSA_OK;
+    if (!o || !lse || !out || !aligned16(o) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+    return launch_cp_merge(o, lse, G, B, H, Dv, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
 dsa_status dsa_swa_decode(const uint16_t *q, const uint16_t *k_ring, const uint16_t *v_ring, const int32_t *seq_lens,
                           int32_t B, int32_t H, int32_t D, int32_t window, float sm_scale, uint16_t *out,
                           dsa_stream_t stream) {

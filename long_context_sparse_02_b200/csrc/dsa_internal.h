@@ -150,6 +150,16 @@ struct AppendArgs {
 };
 dsa_status launch_append(const AppendArgs &a, cudaStream_t st);
 
+// ---- context-parallel decode: joining the ranks' partial results -----------------
+dsa_status launch_cp_candidates(const float *scores, int64_t ld, const int32_t *idx, int B, int K, const int32_t *lo,
+                                float *cs, int32_t *cpos, cudaStream_t st);
+size_t cp_select_workspace_bytes(int G, int B, int K);
+dsa_status launch_cp_select(const float *cs, const int32_t *cpos, int G, int B, int K, const int32_t *lo,
+                            const int32_t *hi, int32_t *idx_g, int32_t *idx_l, void *ws, size_t ws_bytes,
+                            cudaStream_t st);
+dsa_status launch_cp_merge(const uint16_t *o, const float *lse, int G, int B, int H, int Dv, uint16_t *out,
+                           cudaStream_t st);
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace dsa
