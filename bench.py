@@ -399,6 +399,7 @@ def run_native(args):
             res.update(long_context_leg(args, flush, peaks))
             res["prefill_layer"] = prefill_layer_leg(args, flush, peaks)
             res["tiny_prefill"] = tiny_layer_leg(args, flush)
+            res["mxfp8_decode"] = mx_leg(args, flush, peaks)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -800,6 +801,63 @@ def prefill_layer_leg(args, flush, peaks, T=32768, reps=3):
                                           "sample": f"rows {rows.tolist()} timed per stage, scaled by keys scored "
                                                     f"and rows attended", **host_cpu()}
         del q, kv, gate, out, idx, ws
+        torch.cuda.empty_cache()
+        return res
+    except Exception as e:
+        return {"error": f"{type(e).__name__}: {e}"[:300]}
+
+
+def mx_leg(args, flush, peaks, steps=100):
+    """MXFP8 indexer operands at the headline's shape (8 x 131072, 32x128):
+    the indexer alone against HBM (keys 128 B + 4 scale bytes per key read,
+    4 B of score written, plus the queries and their scales) and the decode
+    layer with them.  A failure is recorded, not raised."""
+    import numpy as np
+    import torch
+    from long_context_sparse_02_b200 import _lib, synth
+    from long_context_sparse_02_b200.runtime import LayerOnDevice, to_dev
+    try:
+        c = synth.decode_128k(args.seed + 31)
+        r1, r2 = [np.random.default_rng(s) for s in np.random.SeedSequence(args.seed + 32).spawn(2)]
+        c.q_idx, q_sc = synth.mx_dyadic(r1, c.q_idx.shape)
+        c.k_cache, k_sc = synth.mx_dyadic(r2, c.k_cache.shape)
+        lay = LayerOnDevice(c, decode=True)
+        qs, ks = to_dev(q_sc), to_dev(k_sc)
+        la = _lib.layer_args(_lib.MODE_DECODE, lay.q_idx, lay.w, lay.k_cache, lay.q, lay.kv_cache, lay.gate, lay.pg,
+                             None, None, c.K, c.Dv, c.sm_scale, lay.max_len, lay.out, lay.idx, None, qs, ks)
+        ws = torch.zeros(_lib.layer_workspace_bytes(la), dtype=torch.uint8, device="cuda")
+        scores = torch.empty((c.T, lay.max_len), dtype=torch.float32, device="cuda")
+
+        def timed(fn):
+            for _ in range(5):
+                flush.zero_()
+                fn()
+            tot = 0.0
+            for _ in range(steps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize()
+                tot += e0.elapsed_time(e1)
+            return tot / steps
+
+        idx_ms = timed(lambda: _lib.indexer_scores_mx(lay.q_idx, qs, lay.w, lay.k_cache, ks, lay.pg, None, None,
+                                                      lay.max_len, scores))
+        layer_ms = timed(lambda: _lib.layer_forward(la, ws))
+        L, B, HI, DI = int(c.seq_lens[0]), c.T, c.HI, c.DI
+        nbytes = B * L * (DI + DI // 32 + 4) + B * HI * (DI + DI // 32 + 4)
+        gbs = nbytes / (idx_ms * 1e-3) / 1e9
+        hbm = float(peaks["hbm_gbs"])
+        res = {"workload": f"{c.name}_mxfp8",
+               "indexer": {"us": round(idx_ms * 1e3, 2), "algorithmic_bytes": nbytes, "achieved_gbs": round(gbs, 1),
+                           "peak": hbm, "frac_of_hbm": round(gbs / hbm, 4)},
+               "layer": {"us_per_step": round(layer_ms * 1e3, 2), "tokens_per_s": round(B / (layer_ms * 1e-3), 1)}}
+        err = _lib.device_error(reset=True)
+        if err:
+            res["device_error"] = hex(err)
+        del lay, ws, scores
         torch.cuda.empty_cache()
         return res
     except Exception as e:

@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-#define DSA_ABI_VERSION 1
+#define DSA_ABI_VERSION 2
 
 typedef struct CUstream_st *dsa_stream_t; /* same handle as cudaStream_t */
 
@@ -96,6 +96,22 @@ dsa_status dsa_indexer_scores(const uint8_t *q_idx, const float *w,
                               const int32_t *q_seq, const int32_t *q_pos,
                               int32_t T, int32_t HI, int32_t DI, int32_t max_len,
                               float *scores, int64_t ld, dsa_stream_t stream);
+
+/* ---- stage 1 with MXFP8 operands ------------------------------------------------
+ * "Open-Weight Deployment of an Ultra-Large Sparse Model", §1 and §3:
+ * activations in MXFP8, read as the OCP microscaling format.  The same score
+ * as dsa_indexer_scores with qI = q_idx * 2^(q_scales - 127) and kI =
+ * k_idx_cache * 2^(k_scales - 127), one E8M0 scale code per 32 consecutive
+ * elements along DI (code 255 is NaN and out of contract):
+ *   q_scales device uint8 [T, HI, DI/32]; k_scales device uint8
+ *   [num_pages, 64, DI/32] (the key cache's row layout); both 4-byte aligned.
+ * Block-scaled tensor-core MMAs; fp32 accumulation.  Supported: DI == 128,
+ * HI in {16, 32}, T <= 1024.  Needs no workspace. */
+dsa_status dsa_indexer_scores_mx(const uint8_t *q_idx, const uint8_t *q_scales, const float *w,
+                                 const uint8_t *k_idx_cache, const uint8_t *k_scales,
+                                 const dsa_paged *pg, const int32_t *q_seq, const int32_t *q_pos,
+                                 int32_t T, int32_t HI, int32_t DI, int32_t max_len,
+                                 float *scores, int64_t ld, dsa_stream_t stream);
 
 /* ---- stage 2: top-K --------------------------------------------------------
  * For each row r: among positions 0 <= s < row_len[r], keep the K largest
@@ -209,6 +225,10 @@ typedef struct {
     uint16_t *out;              /* device bf16 [T, H, Dv] */
     int32_t *idx_out;           /* device int32 [T, K] or NULL */
     float *lse;                 /* device fp32 [T, H] or NULL */
+    /* MXFP8 indexer operands (dsa_indexer_scores_mx): both NULL for per-tensor
+     * FP8, or both set (DI == 128, HI in {16, 32}, T <= 1024) */
+    const uint8_t *q_idx_scales; /* device uint8 [T, HI, DI/32] */
+    const uint8_t *k_idx_scales; /* device uint8 [num_pages, 64, DI/32] */
 } dsa_layer_args;
 
 /* Workspace: (decode, or T <= 64) a per-query histogram of the indexer scores, then the
@@ -310,6 +330,21 @@ dsa_status dsa_cp_select(const float *cand_score, const int32_t *cand_pos, int32
  *   o and out 16-byte aligned. */
 dsa_status dsa_cp_lse_merge(const uint16_t *o, const float *lse, int32_t G, int32_t B,
                             int32_t H, int32_t Dv, uint16_t *out, dsa_stream_t stream);
+
+/* ---- the step before the layer, MXFP8 keys -------------------------------------------
+ * As dsa_append_kv, with the indexer keys stored in MXFP8 ("Open-Weight
+ * Deployment of an Ultra-Large Sparse Model", §1 and §3), read as the OCP
+ * microscaling format: each 32 consecutive elements x of a key row share the
+ * scale code c = clamp(floor(log2 max|x|) - 8, -127, 127) + 127 (an all-zero
+ * block: c = 0), stored in k_scales at the row's position; the elements
+ * become e4m3(x * 2^(127 - c)), to the nearest code with ties to the even
+ * mantissa, saturating to +-448.
+ *   k_scales device uint8 [num_pages, 64, DI/32].  Supported: DI in {64, 128};
+ *   Dqk a multiple of 8, at most 768.  Needs no workspace. */
+dsa_status dsa_append_kv_mx(const uint16_t *k_new, const uint16_t *latent_new,
+                            const int32_t *tok_seq, const int32_t *tok_pos, const dsa_paged *pg,
+                            int32_t n, int32_t DI, int32_t Dqk, uint8_t *k_idx_cache,
+                            uint8_t *k_scales, uint16_t *kv_cache, dsa_stream_t stream);
 
 /* ---- housekeeping ---------------------------------------------------------------- */
 const char *dsa_status_string(dsa_status s);

@@ -49,7 +49,7 @@ class LayerArgs(ctypes.Structure):
     _fields_ = [("mode", I32), ("q_idx", P), ("w", P), ("k_idx_cache", P), ("q", P), ("kv_cache", P),
                 ("gate", P), ("pg", Paged), ("q_seq", P), ("q_pos", P), ("T", I32), ("HI", I32), ("DI", I32),
                 ("K", I32), ("H", I32), ("Dqk", I32), ("Dv", I32), ("max_len", I32), ("sm_scale", F32),
-                ("out", P), ("idx_out", P), ("lse", P)]
+                ("out", P), ("idx_out", P), ("lse", P), ("q_idx_scales", P), ("k_idx_scales", P)]
 
 
 lib.dsa_abi_version.restype = I32
@@ -60,6 +60,10 @@ lib.dsa_device_error.restype = ctypes.c_int
 lib.dsa_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), I32]
 lib.dsa_indexer_scores.restype = ctypes.c_int
 lib.dsa_indexer_scores.argtypes = [P, P, P, ctypes.POINTER(Paged), P, P, I32, I32, I32, I32, P, I64, P]
+lib.dsa_indexer_scores_mx.restype = ctypes.c_int
+lib.dsa_indexer_scores_mx.argtypes = [P, P, P, P, P, ctypes.POINTER(Paged), P, P, I32, I32, I32, I32, P, I64, P]
+lib.dsa_append_kv_mx.restype = ctypes.c_int
+lib.dsa_append_kv_mx.argtypes = [P, P, P, P, ctypes.POINTER(Paged), I32, I32, I32, P, P, P, P]
 lib.dsa_topk_workspace_bytes.restype = SZ
 lib.dsa_topk_workspace_bytes.argtypes = [I32, I32, I32]
 lib.dsa_topk.restype = ctypes.c_int
@@ -96,7 +100,8 @@ lib.dsa_cp_lse_merge.argtypes = [P, P, I32, I32, I32, I32, P, P]
 lib.dsa_swa_decode.restype = ctypes.c_int
 lib.dsa_swa_decode.argtypes = [P, P, P, P, I32, I32, I32, I32, F32, P, P]
 
-EXPORTS = ["dsa_abi_version", "dsa_status_string", "dsa_device_error", "dsa_indexer_scores",
+EXPORTS = ["dsa_abi_version", "dsa_status_string", "dsa_device_error", "dsa_indexer_scores", "dsa_indexer_scores_mx",
+           "dsa_append_kv_mx",
            "dsa_topk_workspace_bytes", "dsa_topk", "dsa_topk_hist_workspace_bytes", "dsa_topk_hist", "dsa_topk_static", "dsa_sparse_attn_workspace_bytes",
            "dsa_sparse_attn",
            "dsa_layer_workspace_bytes", "dsa_layer_forward", "dsa_layer_forward_profiled",
@@ -208,7 +213,8 @@ def sparse_attn(q, kv_cache, pg: Paged, q_seq, idx, gate, sm_scale: float, Dv: i
 
 
 def layer_args(mode, q_idx, w, k_cache, q, kv_cache, gate, pg: Paged, q_seq, q_pos, K: int, Dv: int,
-               sm_scale: float, max_len: int, out, idx_out=None, lse=None) -> LayerArgs:
+               sm_scale: float, max_len: int, out, idx_out=None, lse=None, q_scales=None,
+               k_scales=None) -> LayerArgs:
     T, HI, DI = q_idx.shape
     _, H, Dqk = q.shape
     a = LayerArgs(int(mode), _ptr(q_idx, torch.uint8, "q_idx"), _ptr(w, torch.float32, "w"),
@@ -217,9 +223,10 @@ def layer_args(mode, q_idx, w, k_cache, q, kv_cache, gate, pg: Paged, q_seq, q_p
                      _ptr(q_seq, torch.int32, "q_seq", True), _ptr(q_pos, torch.int32, "q_pos", True),
                      T, HI, DI, int(K), H, Dqk, int(Dv), int(max_len), float(sm_scale),
                      _ptr(out, torch.bfloat16, "out"), _ptr(idx_out, torch.int32, "idx_out", True),
-                     _ptr(lse, torch.float32, "lse", True))
+                     _ptr(lse, torch.float32, "lse", True), _ptr(q_scales, torch.uint8, "q_scales", True),
+                     _ptr(k_scales, torch.uint8, "k_scales", True))
     a._tensors = (q_idx, w, k_cache, q, kv_cache, gate, getattr(pg, "_tensors", None), q_seq, q_pos, out, idx_out,
-                  lse)
+                  lse, q_scales, k_scales)
     return a
 
 
@@ -306,3 +313,27 @@ def cp_lse_merge(o, lse, out=None):
         _ptr(o, torch.bfloat16, "o"), _ptr(lse, torch.float32, "lse"), G, B, H, Dv, _ptr(out, torch.bfloat16, "out"),
         _stream()))
     return out
+
+
+def indexer_scores_mx(q_idx, q_scales, w, k_cache, k_scales, pg: Paged, q_seq, q_pos, max_len: int, scores):
+    """MXFP8 indexer: q_idx uint8 [T,HI,DI] and q_scales uint8 [T,HI,DI/32]; k_cache uint8 [pages,64,DI] and
+    k_scales uint8 [pages,64,DI/32]; w fp32 [T,HI]; scores fp32 [T, ld]."""
+    T, HI, DI = q_idx.shape
+    _check("dsa_indexer_scores_mx", lib.dsa_indexer_scores_mx(
+        _ptr(q_idx, torch.uint8, "q_idx"), _ptr(q_scales, torch.uint8, "q_scales"), _ptr(w, torch.float32, "w"),
+        _ptr(k_cache, torch.uint8, "k_cache"), _ptr(k_scales, torch.uint8, "k_scales"), ctypes.byref(pg),
+        _ptr(q_seq, torch.int32, "q_seq", True), _ptr(q_pos, torch.int32, "q_pos", True), T, HI, DI, int(max_len),
+        _ptr(scores, torch.float32, "scores"), int(scores.shape[1]), _stream()))
+    return scores
+
+
+def append_kv_mx(k_new, latent_new, tok_seq, tok_pos, pg: Paged, k_cache, k_scales, kv_cache):
+    """MXFP8 append: k_new bf16 [n, DI]; latent_new bf16 [n, Dqk] or None; k_cache uint8 [pages, 64, DI],
+    k_scales uint8 [pages, 64, DI/32] and kv_cache bf16 [pages, 64, Dqk], written in place."""
+    n, DI = k_new.shape
+    Dqk = int(kv_cache.shape[-1]) if kv_cache is not None else 0
+    _check("dsa_append_kv_mx", lib.dsa_append_kv_mx(
+        _ptr(k_new, torch.bfloat16, "k_new"), _ptr(latent_new, torch.bfloat16, "latent_new", True),
+        _ptr(tok_seq, torch.int32, "tok_seq"), _ptr(tok_pos, torch.int32, "tok_pos"), ctypes.byref(pg), n, DI, Dqk,
+        _ptr(k_cache, torch.uint8, "k_cache"), _ptr(k_scales, torch.uint8, "k_scales"),
+        _ptr(kv_cache, torch.bfloat16, "kv_cache", True), _stream()))

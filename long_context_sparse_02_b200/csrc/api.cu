@@ -207,6 +207,23 @@ dsa_status dsa_indexer_scores(const uint8_t *q_idx, const float *w, const uint8_
     return launch_indexer(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+dsa_status dsa_indexer_scores_mx(const uint8_t *q_idx, const uint8_t *q_scales, const float *w,
+                                 const uint8_t *k_idx_cache, const uint8_t *k_scales, const dsa_paged *pg,
+                                 const int32_t *q_seq, const int32_t *q_pos, int32_t T, int32_t HI, int32_t DI,
+                                 int32_t max_len, float *scores, int64_t ld, dsa_stream_t stream) {
+    if (T < 0 || !paged_ok(pg) || max_len < 1 || ld < max_len) return DSA_ERR_INVALID_ARG;
+    if ((q_seq == nullptr) != (q_pos == nullptr)) return DSA_ERR_INVALID_ARG;
+    if (!q_seq && T > pg->num_seqs) return DSA_ERR_INVALID_ARG;
+    if ((HI != 16 && HI != 32) || DI != 128 || T > 1024) return DSA_ERR_UNSUPPORTED;
+    if (T == 0) return DSA_OK;
+    if (!q_idx || !q_scales || !w || !k_idx_cache || !k_scales || !scores) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q_idx) || !aligned16(k_idx_cache) || (reinterpret_cast<uintptr_t>(q_scales) & 3u) ||
+        (reinterpret_cast<uintptr_t>(k_scales) & 3u))
+        return DSA_ERR_INVALID_ARG;
+    IndexerArgs a{q_idx, w, k_idx_cache, paged_dev(pg), q_seq, q_pos, T, HI, DI, max_len, scores, ld};
+    return launch_indexer_mx(a, q_scales, k_scales, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t dsa_topk_workspace_bytes(int32_t R, int32_t K, int32_t max_row_len) {
     if (R <= 0 || K <= 0 || max_row_len <= 0) return 0;
     return topk_workspace_bytes(R, K, max_row_len);
@@ -305,6 +322,9 @@ dsa_status layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes, dsa
     if (!aligned16(a->q_idx) || !aligned16(a->k_idx_cache) || !aligned16(a->q) || !aligned16(a->kv_cache) ||
         !aligned16(a->out))
         return DSA_ERR_INVALID_ARG;
+    const bool mx = a->q_idx_scales || a->k_idx_scales;
+    if (mx && (!a->q_idx_scales || !a->k_idx_scales)) return DSA_ERR_INVALID_ARG;
+    if (mx && (a->DI != 128 || (a->HI != 16 && a->HI != 32) || a->T > 1024)) return DSA_ERR_UNSUPPORTED;
     LayerWs lw = carve_layer(a, ws);
     if (!ws || ws_bytes < lw.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return DSA_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -315,7 +335,7 @@ dsa_status layer_forward(const dsa_layer_args *a, void *ws, size_t ws_bytes, dsa
                    hist_mode(a) ? static_cast<uint32_t *>(lw.topk_ws) : nullptr,
                    hist_mode(a) ? topk_hist_zero_words(a->T) : 0};
     if (!mark(0)) return DSA_ERR_CUDA;
-    dsa_status s = launch_indexer(ia, st);
+    dsa_status s = mx ? launch_indexer_mx(ia, a->q_idx_scales, a->k_idx_scales, st) : launch_indexer(ia, st);
     if (s != DSA_OK) return s;
     if (!mark(1)) return DSA_ERR_CUDA;
     TopkArgs ta{lw.scores, ld, decode ? a->pg.seq_lens : a->q_pos,
@@ -405,6 +425,21 @@ dsa_status dsa_cp_lse_merge(const uint16_t *o, const float *lse, int32_t G, int3
     if (B == 0) return DSA_OK;
     if (!o || !lse || !out || !aligned16(o) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
     return launch_cp_merge(o, lse, G, B, H, Dv, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_append_kv_mx(const uint16_t *k_new, const uint16_t *latent_new, const int32_t *tok_seq,
+                            const int32_t *tok_pos, const dsa_paged *pg, int32_t n, int32_t DI, int32_t Dqk,
+                            uint8_t *k_idx_cache, uint8_t *k_scales, uint16_t *kv_cache, dsa_stream_t stream) {
+    if (n < 0 || !paged_ok(pg)) return DSA_ERR_INVALID_ARG;
+    if ((DI != 64 && DI != 128) || (latent_new && (Dqk < 8 || Dqk % 8 || Dqk > 768))) return DSA_ERR_UNSUPPORTED;
+    if (n == 0) return DSA_OK;
+    if (!k_new || !tok_seq || !tok_pos || !k_idx_cache || !k_scales || (latent_new && !kv_cache))
+        return DSA_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(k_idx_cache) || (latent_new && (!aligned16(latent_new) || !aligned16(kv_cache))))
+        return DSA_ERR_INVALID_ARG;
+    AppendArgs a{k_new, latent_new, tok_seq, tok_pos, paged_dev(pg), n, DI, latent_new ? Dqk : 0, 1.f,
+                 k_idx_cache, kv_cache};
+    return launch_append_mx(a, k_scales, reinterpret_cast<cudaStream_t>(stream));
 }
 
 dsa_status dsa_swa_decode(const uint16_t *q, const uint16_t *k_ring, const uint16_t *v_ring, const int32_t *seq_lens,

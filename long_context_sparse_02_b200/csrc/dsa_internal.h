@@ -65,6 +65,10 @@ dsa_status launch_indexer(const IndexerArgs &a, cudaStream_t st);
 // Few explicit queries (T <= 64, 16 or 32 heads x 128): consecutive queries of
 // one sequence share each key tile.  launch_indexer routes them here.
 bool indexer_group_eligible(const IndexerArgs &a);
+// MXFP8 operands: E8M0 scales, q_scales [T, HI, DI/32], k_scales [pages, 64, DI/32]
+// (DI = 128, HI in {16, 32}).
+dsa_status launch_indexer_mx(const IndexerArgs &a, const uint8_t *q_scales, const uint8_t *k_scales,
+                             cudaStream_t st);
 dsa_status launch_indexer_group(const IndexerArgs &a, cudaStream_t st);
 
 // ---- top-K ---------------------------------------------------------------------
@@ -149,6 +153,8 @@ struct AppendArgs {
     uint16_t *kv_cache;
 };
 dsa_status launch_append(const AppendArgs &a, cudaStream_t st);
+// MXFP8 keys: codes into k_cache, one E8M0 scale per 32 elements into k_scales [pages, 64, DI/32].
+dsa_status launch_append_mx(const AppendArgs &a, uint8_t *k_scales, cudaStream_t st);
 
 // ---- context-parallel decode: joining the ranks' partial results -----------------
 dsa_status launch_cp_candidates(const float *scores, int64_t ld, const int32_t *idx, int B, int K, const int32_t *lo,

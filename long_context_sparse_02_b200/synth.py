@@ -47,6 +47,19 @@ def dyadic_e4m3(rng: np.random.Generator, shape, lo: int = -4, hi: int = 4) -> n
     return f32_to_e4m3_bits(n.astype(np.float32) / 16.0)
 
 
+def mx_dyadic(rng: np.random.Generator, shape, lo_code: int = 117, hi_code: int = 132):
+    """MXFP8 operands whose decoded values are the dyadic indexer values
+    n * 2^-4, n in [-4, 4]: each 32-element block along the last axis draws a
+    scale code c in [lo_code, hi_code] and stores the elements as E4M3 codes
+    of n * 2^-4 / 2^(c - 127) (exact in E4M3 for codes 117..132).  Returns
+    (element codes uint8 [..., n], scale codes uint8 [..., n/32])."""
+    shape = tuple(shape)
+    n = rng.integers(-4, 5, size=shape).astype(np.float32)
+    codes = rng.integers(lo_code, hi_code + 1, size=shape[:-1] + (shape[-1] // 32,)).astype(np.uint8)
+    s = np.repeat(codes.astype(np.int32) - 127, 32, axis=-1)
+    return f32_to_e4m3_bits(np.ldexp(n * np.float32(2.0 ** -4), -s).astype(np.float32)), codes
+
+
 def dyadic_weights(rng: np.random.Generator, shape, signed: bool = False) -> np.ndarray:
     """fp32 weights n * 2^-6, n uniform in [0, 64] (or [-64, 64] when signed)."""
     lo = -64 if signed else 0

@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.lib.dsa_abi_version() == 1
+    assert lib.lib.dsa_abi_version() == 2
     assert lib.lib.dsa_status_string(0) == b"ok"
     assert lib.lib.dsa_status_string(3).startswith(b"workspace")
 
