@@ -222,8 +222,9 @@ def profiled_traffic():
 # ---------------------------------------------------------------- algorithmic work
 
 def decode_bytes(case):
-    """Bytes the decode layer must move (no score round trip), and the indexer
-    kernel's own I/O (its key stream, queries, weights and the scores it writes)."""
+    """Bytes the decode layer must move (no score round trip), and the decode
+    indexer's algorithmic bytes (its key stream, queries and weights: the score
+    round trip is not part of the method)."""
     L = case.seq_lens.astype(float)
     kI = float((L * case.DI).sum())
     qI = case.T * case.HI * case.DI + case.T * case.HI * 4
@@ -233,8 +234,14 @@ def decode_bytes(case):
     gate = case.T * case.H * 2
     out = case.T * case.H * case.Dv * 2
     layer = kI + qI + gather + q + gate + out
-    indexer = kI + qI + float(L.sum()) * 4
+    indexer = kI + qI
     return layer, indexer
+
+
+def score_write_bytes(case):
+    """The fp32 scores the decode indexer writes (one per key): the score
+    round trip, reported beside the algorithmic figure."""
+    return float(case.seq_lens.astype(float).sum()) * 4
 
 
 # nominal B200 peaks, reported beside the measured ones: HBM3e 7.7 TB/s (HGX), dense FP8 4.5 PFLOP/s
@@ -349,12 +356,15 @@ def run_native(args):
     hbm = float(peaks["hbm_gbs"])
     layer_bytes, idx_bytes = decode_bytes(case)
     idx_gbs = idx_bytes / (st["indexer"] * 1e-6) / 1e9
+    io_gbs = (idx_bytes + score_write_bytes(case)) / (st["indexer"] * 1e-6) / 1e9
     traffic, traffic_src = profiled_traffic()
     roofline = {"bound": "hbm", "kernel": "indexer_decode_kernel<128,32> (stage 1 of dsa_layer_forward)",
                 "achieved": round(idx_gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(idx_gbs / hbm, 4),
                 "peak_spec": SPEC_HBM_GBS, "frac_spec": round(idx_gbs / SPEC_HBM_GBS, 4),
                 "traffic": traffic, "traffic_source": traffic_src,
                 "algorithmic_bytes_per_launch": idx_bytes, "launch_us": round(st["indexer"], 2),
+                "with_score_writes": {"bytes_per_launch": idx_bytes + score_write_bytes(case),
+                                      "achieved": round(io_gbs, 1), "frac": round(io_gbs / hbm, 4)},
                 "peak_source": f"hbm_gbs, {peak_src}"}
     step_mean_ms = total_ms / args.steps
     layer_gbs = layer_bytes / (step_mean_ms * 1e-3) / 1e9
@@ -408,10 +418,16 @@ def run_native(args):
 
 
 def e2e_leg(args, lay, flush, stream, _lib):
-    """The same decode step through dsa_layer_forward with the step's inputs
-    coming from pinned host memory and its output going back to it.  The
-    per-step inputs (qI, w, q, gate, seq_lens) sit in one pinned buffer and go
-    over in one copy; the caches stay resident."""
+    """The decode step end to end through dsa_layer_forward: each step's inputs
+    (qI, w, q, gate, seq_lens, in one pinned host buffer) go over in one copy
+    and its output comes back to pinned host memory.  Pipelined as a serving
+    loop runs it: two input and two output buffers; step i+1's upload (one
+    copy stream) and step i-1's download (another) overlap step i's layer on
+    the compute stream, ordered by events.  One event pair spans all K steps
+    (on the download stream, after the last copy); every step streams its
+    134 MB of keys and its gathered rows, more than the 126 MB L2, so nothing
+    stays cached from step to step.  The unpipelined form (copy in, layer,
+    copy out; L2 flushed between steps) is reported beside it."""
     import torch
     K = max(20, args.steps // 2)
     c = lay.case
@@ -421,18 +437,24 @@ def e2e_leg(args, lay, flush, stream, _lib):
         offs.append(off)
         off += (t.numel() * t.element_size() + 255) // 256 * 256
     host_in = torch.empty(off, dtype=torch.uint8).pin_memory()
-    dev_in = torch.empty(off, dtype=torch.uint8, device="cuda")
-    views = []
     for t, o in zip(srcs, offs):
         nb = t.numel() * t.element_size()
         host_in[o:o + nb].copy_(t.reshape(-1).view(torch.uint8).cpu())
-        views.append(dev_in[o:o + nb].view(t.dtype).view(t.shape))
-    pg = _lib.paged(views[4], lay.block_table, c.num_pages, c.page_size)
-    out = torch.empty_like(lay.out)
-    a = _lib.layer_args(_lib.MODE_DECODE, views[0], views[1], lay.k_cache, views[2], lay.kv_cache, views[3], pg,
-                        None, None, c.K, c.Dv, c.sm_scale, lay.max_len, out, lay.idx, None)
-    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    bufs = []
+    for _ in range(2):
+        dev_in = torch.empty(off, dtype=torch.uint8, device="cuda")
+        views = [dev_in[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape) for t, o in zip(srcs, offs)]
+        pg = _lib.paged(views[4], lay.block_table, c.num_pages, c.page_size)
+        out = torch.empty_like(lay.out)
+        a = _lib.layer_args(_lib.MODE_DECODE, views[0], views[1], lay.k_cache, views[2], lay.kv_cache, views[3], pg,
+                            None, None, c.K, c.Dv, c.sm_scale, lay.max_len, out, lay.idx, None)
+        host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        bufs.append((dev_in, a, out, host_out))
+    d2h = bufs[0][3].numel() * bufs[0][3].element_size()
+
+    # unpipelined: one step at a time, L2 flushed between steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K + 3)]
+    dev_in, a, out, host_out = bufs[0]
     for s, e in ev:
         flush.zero_()
         s.record(stream)
@@ -441,14 +463,58 @@ def e2e_leg(args, lay, flush, stream, _lib):
         host_out.copy_(out, non_blocking=True)
         e.record(stream)
     torch.cuda.synchronize()
-    ms = sum(s.elapsed_time(e) for s, e in ev[3:])
+    serial_ms = sum(s.elapsed_time(e) for s, e in ev[3:]) / K
     if not torch.equal(host_out, lay.out.cpu()):
         raise RuntimeError("end-to-end output differs from the device-resident run")
-    d2h = host_out.numel() * host_out.element_size()
-    return {"value": round(c.T * K / (ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": int(off),
-            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms / K, 5),
-            "note": "dsa_layer_forward; the step's inputs (qI, w, q, gate, seq_lens) in one pinned-host->device "
-                    "copy and the output device->pinned-host, inside the events; caches stay resident"}
+
+    # pipelined
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    copied_out = [torch.cuda.Event() for _ in range(2)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def run(n, timed):
+        torch.cuda.synchronize()
+        if timed:
+            t0.record(up)
+        for i in range(n + 1):
+            if i < n:  # upload step i (its buffer is free once step i-2's layer is done)
+                b = i & 1
+                with torch.cuda.stream(up):
+                    if i >= 2:
+                        up.wait_event(done[b])
+                    bufs[b][0].copy_(host_in, non_blocking=True)
+                    in_ready[b].record(up)
+                stream.wait_event(in_ready[b])
+                if i >= 2:
+                    stream.wait_event(copied_out[b])  # its output buffer has been read back
+                _lib.layer_forward(bufs[b][1], lay.ws)
+                done[b].record(stream)
+            if i >= 1:  # download step i-1
+                b = (i - 1) & 1
+                with torch.cuda.stream(down):
+                    down.wait_event(done[b])
+                    bufs[b][3].copy_(bufs[b][2], non_blocking=True)
+                    copied_out[b].record(down)
+        if timed:
+            up.wait_stream(down)
+            t1.record(up)
+        torch.cuda.synchronize()
+
+    run(4, False)
+    run(K, True)
+    piped_ms = t0.elapsed_time(t1) / K
+    if not torch.equal(bufs[(K - 1) & 1][3], lay.out.cpu()):
+        raise RuntimeError("pipelined end-to-end output differs from the device-resident run")
+    return {"value": round(c.T / (piped_ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": int(off),
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(piped_ms, 5),
+            "note": "dsa_layer_forward in a pipelined loop: each step's inputs (qI, w, q, gate, seq_lens) one "
+                    "pinned-host->device copy, its output device->pinned-host, uploads and downloads on their own "
+                    "streams overlapping the neighbouring steps' layers; one event pair over all steps; caches "
+                    "stay resident; per-step working set > L2",
+            "serial": {"value": round(c.T / (serial_ms / 1e3), 1), "ms_per_step": round(serial_ms, 5),
+                       "note": "copy in, layer, copy out, one step at a time, L2 flushed between steps"}}
 
 
 def fp8_peak_tflops():

@@ -346,6 +346,18 @@ dsa_status dsa_append_kv_mx(const uint16_t *k_new, const uint16_t *latent_new,
                             int32_t n, int32_t DI, int32_t Dqk, uint8_t *k_idx_cache,
                             uint8_t *k_scales, uint16_t *kv_cache, dsa_stream_t stream);
 
+/* ---- testing the bounded waits ------------------------------------------------------
+ * Every pipeline wait in the kernels gives up after a time limit (1 s),
+ * records DSA_DEVERR_TIMEOUT, lets the CTA's other roles abandon their work,
+ * waits (again with a limit) for its own copies in flight, frees its tensor
+ * memory and returns.  For testing that path without any fault: while `tile`
+ * >= 0, every later launch of the decode indexer (the layer's decode mode and
+ * dsa_indexer_scores without q_seq) leaves flattened tile `tile` -- the
+ * queries' 128-key tiles in order -- unfilled, so the wait on it runs out;
+ * that launch's scores are then incomplete.  -1 turns it off (the default).
+ * Host-side setting, all devices. */
+dsa_status dsa_test_skip_indexer_tile(int64_t tile);
+
 /* ---- housekeeping ---------------------------------------------------------------- */
 const char *dsa_status_string(dsa_status s);
 int32_t dsa_abi_version(void);

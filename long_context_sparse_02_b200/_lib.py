@@ -97,6 +97,8 @@ lib.dsa_cp_select.restype = ctypes.c_int
 lib.dsa_cp_select.argtypes = [P, P, I32, I32, I32, P, P, P, P, P, SZ, P]
 lib.dsa_cp_lse_merge.restype = ctypes.c_int
 lib.dsa_cp_lse_merge.argtypes = [P, P, I32, I32, I32, I32, P, P]
+lib.dsa_test_skip_indexer_tile.restype = ctypes.c_int
+lib.dsa_test_skip_indexer_tile.argtypes = [I64]
 lib.dsa_swa_decode.restype = ctypes.c_int
 lib.dsa_swa_decode.argtypes = [P, P, P, P, I32, I32, I32, I32, F32, P, P]
 
@@ -106,7 +108,8 @@ EXPORTS = ["dsa_abi_version", "dsa_status_string", "dsa_device_error", "dsa_inde
            "dsa_sparse_attn",
            "dsa_layer_workspace_bytes", "dsa_layer_forward", "dsa_layer_forward_profiled",
            "dsa_layer_kernel_launches", "dsa_swa_decode", "dsa_append_kv", "dsa_cp_candidates",
-           "dsa_cp_select_workspace_bytes", "dsa_cp_select", "dsa_cp_lse_merge"]
+           "dsa_cp_select_workspace_bytes", "dsa_cp_select", "dsa_cp_lse_merge",
+           "dsa_test_skip_indexer_tile"]
 
 
 def _check(fn: str, status: int):

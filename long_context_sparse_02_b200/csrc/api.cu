@@ -4,6 +4,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <utility>
 #include <vector>
@@ -33,6 +34,11 @@ EncodeTiled g_encode = nullptr;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 }  // namespace
+
+namespace {
+std::atomic<int64_t> g_test_skip_tile{-1};
+}
+int64_t test_skip_tile() { return g_test_skip_tile.load(std::memory_order_relaxed); }
 
 const DeviceInfo *current_device() {
     int d = -1;
@@ -169,6 +175,12 @@ LayerWs carve_layer(const dsa_layer_args *a, void *ws) {
 extern "C" {
 
 int32_t dsa_abi_version(void) { return DSA_ABI_VERSION; }
+
+dsa_status dsa_test_skip_indexer_tile(int64_t tile) {
+    if (tile < -1) return DSA_ERR_INVALID_ARG;
+    g_test_skip_tile.store(tile, std::memory_order_relaxed);
+    return DSA_OK;
+}
 
 const char *dsa_status_string(dsa_status s) {
     switch (s) {

@@ -65,6 +65,9 @@ dsa_status launch_indexer(const IndexerArgs &a, cudaStream_t st);
 // Few explicit queries (T <= 64, 16 or 32 heads x 128): consecutive queries of
 // one sequence share each key tile.  launch_indexer routes them here.
 bool indexer_group_eligible(const IndexerArgs &a);
+// The flattened tile (all queries' 128-key tiles in order) that later
+// decode-indexer launches leave unfilled, -1 = none: dsa_test_skip_indexer_tile.
+int64_t test_skip_tile();
 // MXFP8 operands: E8M0 scales, q_scales [T, HI, DI/32], k_scales [pages, 64, DI/32]
 // (DI = 128, HI in {16, 32}).
 dsa_status launch_indexer_mx(const IndexerArgs &a, const uint8_t *q_scales, const uint8_t *k_scales,

@@ -233,7 +233,10 @@ __global__ void __launch_bounds__(DecCfg<DI, NH>::THREADS, DecCfg<DI, NH>::CTAS_
                     if (ok && mbar_wait(&empty[s], ph ^ 1, p.err, abort_flag)) {
                         uint8_t *A = stages + s * C::A_BYTES;
                         const uint32_t bytes = (pg0 >= 0 ? 64 * DI : 0) + (pg1 >= 0 ? 64 * DI : 0);
-                        if (bytes) {
+                        if (lo + i + 1 == p.test_skip_tile_plus1) {
+                            // testing the bounded waits: this tile is never filled, so the
+                            // MMA's wait on it runs out and the CTA abandons its work
+                        } else if (bytes) {
                             mbar_expect_tx(&full[s], bytes);
                             if (pg0 >= 0) tma_load_2d_hint(A, &kmap, &full[s], 0, pg0 * 64, kpol);
                             if (pg1 >= 0) tma_load_2d_hint(A + 64 * DI, &kmap, &full[s], 0, pg1 * 64, kpol);
@@ -765,7 +768,7 @@ dsa_status launch_indexer(const IndexerArgs &a, cudaStream_t st) {
     if (indexer_group_eligible(a)) return launch_indexer_group(a, st);
     IdxParams p{a.w, a.q_seq, a.q_pos, a.pg, a.T, a.HI, a.max_len, a.scores, a.ld, dev->err,
                 (a.q_seq == nullptr || a.T <= 64) ? a.hist : nullptr,  // the few-query kernel counts
-                a.zero, a.nzero};
+                a.zero, a.nzero, test_skip_tile() + 1};
     const CUtensorMapSwizzle swz = a.DI == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUtensorMap km, qm;
     if (!make_tmap_2d(&km, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.DI, (uint64_t)a.pg.num_pages * 64, a.DI,

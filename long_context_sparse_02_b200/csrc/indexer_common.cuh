@@ -75,6 +75,10 @@ struct IdxParams {
     uint32_t *hist;  // [T][SCORE_HIST_BINS] or NULL (few-query kernels only)
     uint32_t *zero;  // nzero words the grid sets to zero (or NULL)
     int64_t nzero;
+    // testing the bounded waits (decode kernel): flattened tile
+    // test_skip_tile_plus1 - 1 (queries' 128-key tiles in order) is never
+    // filled; 0 = off
+    int64_t test_skip_tile_plus1;
 };
 
 // The grid clears the words the next kernel expects at zero, each CTA a share.

@@ -16,9 +16,11 @@ def _case(seq_lens, HI, DI=128, K=2048, H=128, Dqk=576, Dv=512):
 def test_decode_128k_bytes():
     # layer: keys 8*131072*128 + queries/weights 8*32*(128+4) + gathered rows 8*2048*1152
     #        + q 8*128*1152 + gate 8*128*2 + out 8*128*1024 = 155,356,160
-    # indexer launch: keys + queries/weights + scores 8*131072*4 = 138,445,824
-    layer, indexer = bench.decode_bytes(_case([131072] * 8, HI=32))
-    assert layer == 155_356_160 and indexer == 138_445_824
+    # indexer (algorithmic): keys + queries/weights = 134,251,520; with its 8*131072*4 score writes 138,445,824
+    c = _case([131072] * 8, HI=32)
+    layer, indexer = bench.decode_bytes(c)
+    assert layer == 155_356_160 and indexer == 134_251_520
+    assert indexer + bench.score_write_bytes(c) == 138_445_824
 
 
 def test_decode_1m_bytes():

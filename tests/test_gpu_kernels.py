@@ -403,3 +403,40 @@ def test_append_kv_reports_bad_positions_without_fault(L, orc):
     torch.cuda.synchronize()
     assert L.device_error(reset=True) == 1  # DSA_DEVERR_POSITION: position 100 is past the sequence
     assert (k_cache[0, 5] == 0x38).all() and int(k_cache.sum()) == 0x38 * 128  # only the valid token landed
+
+
+# ------------------------------------------------------------------ bounded waits
+
+def test_timed_out_wait_abandons_the_launch_and_the_next_call_is_exact(L, orc):
+    """A decode-indexer tile that is never filled (dsa_test_skip_indexer_tile):
+    the MMA's wait on it runs out after its limit, the error word reports
+    DSA_DEVERR_TIMEOUT, the launch returns (its CTAs free their tensor memory)
+    and the context stays usable -- the next call, with the tile filled
+    again, is bit-exact."""
+    import time
+    from long_context_sparse_02_b200.runtime import LayerOnDevice
+    c = synth.decode_case(21, [3000, 1200], HI=32, K=256, H=16, Dqk=64, Dv=64)
+    pg = orc.Paged(c.seq_lens, c.block_table, 64, c.num_pages)
+    _, idx, out = orc.layer_forward(c.q_idx, c.w, c.k_cache, c.q, c.kv_cache, c.gate, pg,
+                                    np.arange(2, dtype=np.int32), (c.seq_lens - 1).astype(np.int32), c.K, c.Dv,
+                                    c.sm_scale)
+    lay = LayerOnDevice(c, decode=True)
+    L.device_error(reset=True)
+    try:
+        assert L.lib.dsa_test_skip_indexer_tile(0) == 0
+        t0 = time.perf_counter()
+        lay.forward()
+        torch.cuda.synchronize()
+        dt = time.perf_counter() - t0
+    finally:
+        assert L.lib.dsa_test_skip_indexer_tile(-1) == 0
+    err = L.device_error(reset=True)
+    assert err & L.DEVERR_TIMEOUT, hex(err)
+    assert dt < 10.0, dt  # the waits are bounded: about a second each
+    for _ in range(2):
+        lay.forward()
+        torch.cuda.synchronize()
+        assert L.device_error(reset=True) == 0
+        assert np.array_equal(lay.idx.cpu().numpy(), idx)
+        assert_attn_close(lay.out.float().cpu().numpy().astype(np.float64), out)
+    assert L.lib.dsa_test_skip_indexer_tile(-2) == 1  # out of range: rejected
