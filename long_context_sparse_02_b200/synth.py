@@ -256,7 +256,9 @@ def score_rows(seed: int, R: int, n: int, kind: str = "normal") -> np.ndarray:
     """Synthetic score rows for exercising top-K alone.
     kind: 'normal' (N(0,1) fp32), 'ties' (few distinct values), 'zeros'
     (+0/-0 mix), 'const' (all equal), 'dyadic' (multiples of 2^-14),
-    'outlier' (N(0,1) and one score of 1e30 per row)."""
+    'outlier' (N(0,1) and one score of 1e30 per row), 'narrow'
+    (1 + N(0,1) 2^-20), 'near' / 'cluster' (N(0,1) with an eighth of the
+    row drawn tightly around 1.53: hundreds / thousands of keys per fine bin)."""
     rng = np.random.default_rng(seed)
     if kind == "normal":
         return rng.standard_normal((R, n), dtype=np.float32)
@@ -271,6 +273,14 @@ def score_rows(seed: int, R: int, n: int, kind: str = "normal") -> np.ndarray:
         return np.full((R, n), 1.5, dtype=np.float32)
     if kind == "dyadic":
         return rng.integers(-(1 << 16), 1 << 16, size=(R, n)).astype(np.float32) * (2.0 ** -14)
+    if kind == "narrow":  # 1 + N(0,1) 2^-20: thousands of keys share one fine bin
+        return (1.0 + rng.standard_normal((R, n)) * 2.0 ** -20).astype(np.float32)
+    if kind in ("near", "cluster"):  # N(0,1), an eighth of it moved to 1.53 + N(0,1) 2^-12 (2^-16)
+        v = rng.standard_normal((R, n), dtype=np.float32)
+        m = rng.random((R, n)) < 0.125
+        sd = 2.0 ** -12 if kind == "near" else 2.0 ** -16
+        v[m] = (1.53 + rng.standard_normal(int(m.sum())) * sd).astype(np.float32)
+        return v
     if kind == "outlier":  # N(0,1) with one huge score per row
         v = rng.standard_normal((R, n), dtype=np.float32)
         v[np.arange(R), rng.integers(0, n, size=R)] = 1e30

@@ -136,6 +136,10 @@ TOPK_CASES = [
     (1, 300000, 2048, "zeros"),
     (8, 131072, 2048, "normal"), (4, 4000, 2048, "outlier"), (2, 131072, 2048, "outlier"),
     (80, 70000, 2048, "normal"), (76, 120000, 2048, "dyadic"),
+    # many rows of at most 32768 (prefill): one CTA per row, list in shared memory
+    (300, 32768, 2048, "normal"), (310, 20000, 2048, "ties"), (296, 9000, 512, "dyadic"),
+    (300, 32768, 2048, "narrow"), (300, 32768, 2048, "near"), (300, 32768, 2048, "cluster"), (300, 32768, 2048, "outlier"),
+    (300, 3000, 2048, "zeros"), (300, 9001, 64, "normal"),
 ]
 
 
