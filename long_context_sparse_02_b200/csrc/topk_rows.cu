@@ -14,10 +14,9 @@
 //      the bin, in a 256-bin histogram over the sample's range, that holds
 //      the sample score whose rank is the expected rank of the K-th score
 //      plus four standard deviations;
-//   2. each warp counts its scores >= tf (one ballot per 32 positions), the
-//      counts give each warp its offset, and a second pass over the warp's
-//      range (now in L2) lists them as (position, score) in position order
-//      into shared memory;
+//   2. each warp counts its scores >= tf, the counts give each warp its
+//      offset, and a second pass over the warp's range (now in L2) lists
+//      them as (position, score) in position order into shared memory;
 //   3. a 1024-bin histogram of the listed scores over [tf, sample maximum]
 //      gives the bin F of the K-th score; one pass over the list counts the
 //      entries above F and collects F's few entries, one warp ranks those
@@ -38,19 +37,20 @@ namespace {
 constexpr int TR_THREADS = 256;
 constexpr int TR_WARPS = TR_THREADS / 32;
 constexpr int TR_MINB = 4;     // CTAs per SM
-constexpr int TR_U = 16;       // loads in flight per lane: 16 steps of 32 positions
+constexpr int TR_U = 8;        // loads in flight per lane: 8 steps of 64 positions, a float2 each
 constexpr int TR_MAXN = 32768; // longest row
 constexpr int TR_CAP = 4096;   // listed entries held in shared memory
-constexpr int TR_SMEM = TR_CAP * 8;
+constexpr int TR_SMEM = (TR_CAP + 32) * 8;  // and one scratch entry per lane
 constexpr int TR_RUNS = 64, TR_SAMPLES = TR_RUNS * 32;
-constexpr int TR_BINS = 2048;   // 11 bits per radix level of the exact fallbacks
+constexpr int TR_LB = 11, TR_BINS = 1 << TR_LB;  // bits and bins per radix level of the exact fallbacks
 constexpr int TR_SBINS = 256;   // the sample's histogram
 constexpr int TR_LBINS = 1024;  // the listed scores' histogram
 constexpr int TR_CF = 32;       // entries of the threshold's bin one warp ranks
 constexpr uint32_t TR_PAD = 0xFFFFFFFFu;
 constexpr uint32_t TR_MARK = 0x80000000u;  // set on the position of a kept entry of bin F
+constexpr uint32_t TR_POS = 0xFFFFu;       // a list entry's position bits; its bin sits at bit 16
 static_assert(TR_CAP > TR_SAMPLES, "rows that skip sampling are longer than the sample");
-static_assert((uint32_t)TR_MAXN < TR_MARK, "positions leave the mark bit free");
+static_assert(TR_MAXN <= (int)TR_POS + 1 && TR_LBINS <= 1 << 15, "position, bin and mark share a word");
 
 __device__ __forceinline__ int tr_row_length(const TopkArgs &a, int r, uint32_t *err) {
     int n = a.mode == ROWLEN_QPOS_PLUS_1 ? a.row_len[r] + 1 : a.row_len[r];
@@ -133,7 +133,7 @@ __device__ __forceinline__ int tr_bin(float v, float cap) {
 }
 
 // The rank-th largest (1 <= rank <= count) of the keys get(j), j < count,
-// all within [base, base + span].  Histogram levels of 11 bits over the
+// all within [base, base + span].  Histogram levels of TR_LB bits over the
 // offset key - base; as soon as the chosen bin holds at most 32 keys one warp
 // ranks them.  tau = that key, need = rank - #(keys > tau).
 template <typename Get>
@@ -148,7 +148,7 @@ __device__ __forceinline__ void tr_select(Get get, int count, uint32_t rank, uin
             need = rem;
             return;
         }
-        const int L = H > 11 ? H - 11 : 0;
+        const int L = H > TR_LB ? H - TR_LB : 0;
         const uint32_t bmask = (1u << (H - L)) - 1u;
         for (int i = tid; i < TR_BINS; i += TR_THREADS) sh.hist[i] = 0;
         if (tid == 0) sh.misc[0] = 0, sh.misc[1] = 0, sh.misc[2] = 0, sh.misc[3] = 0, sh.misc[4] = 0, sh.misc[5] = 0;
@@ -242,22 +242,36 @@ __device__ __forceinline__ void tr_compact(Entry entry, int count, uint32_t tau,
     }
 }
 
-// Positions p + 32 u + lane, u < TR_U, of this warp's range [.., hi):
-// one coalesced 128-byte load per u.  Positions at or past hi read as NaN,
-// which no threshold lists (scores are finite).
+// Positions p + 64 u + 2 lane and the next, u < TR_U, of this warp's range
+// [.., hi): one coalesced 256-byte load per u (p is even, so each float2 is
+// aligned).  Positions at or past hi read as NaN, which no threshold lists
+// (scores are finite).
 template <bool FULL>
-__device__ __forceinline__ void tr_load(const float *row, int p, int hi, float (&x)[TR_U]) {
+__device__ __forceinline__ void tr_load(const float *row, int p, int hi, float2 (&x)[TR_U]) {
     const int lane = threadIdx.x & 31;
+    const float nan = __int_as_float(0x7fc00000);
 #pragma unroll
     for (int u = 0; u < TR_U; ++u) {
-        const int q = p + 32 * u + lane;
-        x[u] = (FULL || q < hi) ? __ldcg(row + q) : __int_as_float(0x7fc00000);
+        const int q = p + 64 * u + 2 * lane;
+        if (FULL || q + 1 < hi) {
+            x[u] = __ldcg(reinterpret_cast<const float2 *>(row + q));
+        } else {
+            x[u].x = q < hi ? __ldcg(row + q) : nan;
+            x[u].y = nan;
+        }
     }
 }
 
-__device__ __forceinline__ void tr_load_any(const float *row, int p, int hi, float (&x)[TR_U]) {
-    if (p + 32 * TR_U <= hi) tr_load<true>(row, p, hi, x);
+__device__ __forceinline__ void tr_load_any(const float *row, int p, int hi, float2 (&x)[TR_U]) {
+    if (p + 64 * TR_U <= hi) tr_load<true>(row, p, hi, x);
     else tr_load<false>(row, p, hi, x);
+}
+
+// *p = v where c holds, as one predicated store rather than a branch.
+__device__ __forceinline__ void tr_store_if(bool c, int32_t *p, uint32_t v) {
+    asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t@q st.global.b32 [%1], %2;\n\t}" ::"r"((uint32_t)c),
+                 "l"(p), "r"(v)
+                 : "memory");
 }
 
 // Top-K of the listed entries (K <= listed <= TR_CAP, every score >= lo):
@@ -268,11 +282,15 @@ __device__ __forceinline__ bool tr_finish(uint2 *list, int listed, int K, float 
                                           int32_t *out) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float scale = tr_scale(lo, hi, TR_LBINS);
-    auto bin = [&](uint32_t xbits) { return tr_bin((__uint_as_float(xbits) - lo) * scale, (float)(TR_LBINS - 1)); };
     for (int i = tid; i < TR_LBINS; i += TR_THREADS) sh.hist[i] = 0;
     if (tid == 0) sh.misc[0] = 0, sh.misc[1] = 0, sh.misc[2] = 0, sh.misc[3] = 0;
     __syncthreads();
-    for (int j = tid; j < listed; j += TR_THREADS) atomicAdd(&sh.hist[bin(list[j].y)], 1u);
+    for (int j = tid; j < listed; j += TR_THREADS) {  // each entry keeps its bin for the passes below
+        const uint2 e = list[j];
+        const int bn = tr_bin((__uint_as_float(e.y) - lo) * scale, (float)(TR_LBINS - 1));
+        atomicAdd(&sh.hist[bn], 1u);
+        list[j].x = (e.x & TR_POS) | ((uint32_t)bn << 16);
+    }
     __syncthreads();
     tr_pick<TR_LBINS>(sh.hist, (uint32_t)K, sh.ws, sh.misc);
     const int F = (int)sh.misc[0];
@@ -286,8 +304,8 @@ __device__ __forceinline__ bool tr_finish(uint2 *list, int listed, int K, float 
     uint32_t g = 0;
     for (int j0 = w0; j0 < w1; j0 += 32) {
         const int j = j0 + lane;
-        const uint32_t xb = j < w1 ? list[j].y : 0u;
-        const int bn = j < w1 ? bin(xb) : -1;
+        const uint2 e = j < w1 ? list[j] : make_uint2(0u, 0u);
+        const int bn = j < w1 ? (int)((e.x >> 16) & (TR_LBINS - 1)) : -1;
         g += __popc(__ballot_sync(0xffffffffu, bn > F));
         const uint32_t hm = __ballot_sync(0xffffffffu, bn == F);
         if (hm) {
@@ -295,7 +313,7 @@ __device__ __forceinline__ bool tr_finish(uint2 *list, int listed, int K, float 
             if (lane == 0) b0 = atomicAdd(&sh.misc[3], (uint32_t)__popc(hm));
             b0 = __shfl_sync(0xffffffffu, b0, 0);
             const uint32_t slot = b0 + __popc(hm & lt);
-            if (bn == F && slot < (uint32_t)TR_CF) sh.cf_x[slot] = __uint_as_float(xb), sh.cf_j[slot] = (uint32_t)j;
+            if (bn == F && slot < (uint32_t)TR_CF) sh.cf_x[slot] = __uint_as_float(e.y), sh.cf_j[slot] = (uint32_t)j;
         }
     }
     if (lane == 0) sh.ws[warp] = g;
@@ -324,12 +342,12 @@ __device__ __forceinline__ bool tr_finish(uint2 *list, int listed, int K, float 
     for (int w = 0; w < TR_WARPS; ++w) base += w < warp ? sh.ws[w] : 0u;
     for (int j0 = w0; j0 < w1; j0 += 32) {
         const int j = j0 + lane;
-        const uint2 e = j < w1 ? list[j] : make_uint2(0u, 0u);
-        const int bn = j < w1 ? bin(e.y) : -1;
-        const bool keep = bn > F || (bn == F && (e.x & TR_MARK));
+        const uint32_t ex = j < w1 ? list[j].x : 0u;
+        const int bn = j < w1 ? (int)((ex >> 16) & (TR_LBINS - 1)) : -1;
+        const bool keep = bn > F || (bn == F && (ex & TR_MARK));
         const uint32_t km = __ballot_sync(0xffffffffu, keep);
         const uint32_t slot = base + __popc(km & lt);
-        if (keep && slot < (uint32_t)K) out[slot] = (int32_t)(e.x & ~TR_MARK);
+        tr_store_if(keep && slot < (uint32_t)K, out + slot, ex & TR_POS);
         base += __popc(km);
     }
     return true;
@@ -352,7 +370,7 @@ __device__ __forceinline__ void tr_range(float &lo, float &hi, uint32_t *ws) {
 
 __global__ void __launch_bounds__(TR_THREADS, TR_MINB) topk_rows_kernel(const TopkArgs a, uint32_t *err) {
     __shared__ TrShared sh;
-    extern __shared__ uint2 sh_list[];  // [TR_CAP] (position, score bits), position order
+    extern __shared__ uint2 sh_list[];  // [TR_CAP] (position, score bits), position order; [32] scratch
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int r = blockIdx.x, K = a.K;
     pdl_trigger();
@@ -378,9 +396,9 @@ __global__ void __launch_bounds__(TR_THREADS, TR_MINB) topk_rows_kernel(const To
         listed = (uint32_t)n;
     } else {
         // this warp's range; its first loads are in flight while the threshold is chosen
-        const int span = (n + TR_THREADS - 1) / TR_THREADS * 32;
+        const int span = (n + 2 * TR_THREADS - 1) / (2 * TR_THREADS) * 64;
         const int wlo = min(n, warp * span), whi = min(n, wlo + span);
-        float x[TR_U];
+        float2 x[TR_U];
         tr_load_any(row, wlo, whi, x);
 
         // ---- 1. the list's threshold tf from the sample
@@ -397,26 +415,27 @@ __global__ void __launch_bounds__(TR_THREADS, TR_MINB) topk_rows_kernel(const To
         if (tid == 0) sh.misc[0] = 0;
         tr_range(lo, hi, sh.ws);
         const float scale = tr_scale(lo, hi, TR_SBINS);
+        const float width = (hi - lo) * (1.f / TR_SBINS);
 #pragma unroll
         for (int i = 0; i < PER; ++i) atomicAdd(&sh.hist[tr_bin((sv[i] - lo) * scale, (float)(TR_SBINS - 1))], 1u);
         __syncthreads();
         // the expected rank of the K-th score among the samples, plus four standard deviations
-        const float q = (float)K / (float)n, m = (float)TR_SAMPLES;
-        const int s = min(TR_SAMPLES, (int)ceilf(q * m + 4.f * sqrtf(m * q * (1.f - q))) + 1);
+        const float q = __fdividef((float)K, (float)n), m = (float)TR_SAMPLES;
+        const int s = min(TR_SAMPLES, (int)(q * m + 4.f * sqrtf(m * q * (1.f - q))) + 2);
         tr_pick<TR_SBINS>(sh.hist, (uint32_t)s, sh.ws, sh.misc);
-        // a lower edge at or below the bin's least score; rounding cannot lift it above a listed score that
-        // the count below finds, and the count alone decides what is listed
-        const float tf = scale > 0.f ? lo + (float)sh.misc[0] / scale : lo;
+        // any tf will do: what is listed is decided by the comparisons below alone
+        const float tf = scale > 0.f ? fmaf((float)sh.misc[0], width, lo) : lo;
 
         // ---- 2. count this warp's scores >= tf, then list them at the warp's offset
         uint32_t cw = 0;
         for (int p = wlo;;) {
 #pragma unroll
-            for (int u = 0; u < TR_U; ++u) cw += __popc(__ballot_sync(0xffffffffu, x[u] >= tf));
-            p += 32 * TR_U;
+            for (int u = 0; u < TR_U; ++u) cw += (x[u].x >= tf ? 1u : 0u) + (x[u].y >= tf ? 1u : 0u);
+            p += 64 * TR_U;
             if (p >= whi) break;
             tr_load_any(row, p, whi, x);
         }
+        cw = __reduce_add_sync(0xffffffffu, cw);
         if (lane == 0) sh.ws[warp] = cw;
         __syncthreads();
         uint32_t o = 0;
@@ -427,14 +446,20 @@ __global__ void __launch_bounds__(TR_THREADS, TR_MINB) topk_rows_kernel(const To
         }
         if (listed >= (uint32_t)K && listed <= (uint32_t)TR_CAP) {
             const uint32_t lt = (1u << lane) - 1u;
-            for (int p = wlo; p < whi; p += 32 * TR_U) {
+            for (int p = wlo; p < whi; p += 64 * TR_U) {
                 tr_load_any(row, p, whi, x);
 #pragma unroll
                 for (int u = 0; u < TR_U; ++u) {
-                    const bool in = x[u] >= tf;
-                    const uint32_t m = __ballot_sync(0xffffffffu, in);
-                    if (in) sh_list[o + __popc(m & lt)] = make_uint2((uint32_t)(p + 32 * u + lane), __float_as_uint(x[u]));
-                    o += __popc(m);
+                    // order within the step: lane, then the lane's two positions
+                    const bool i0 = x[u].x >= tf, i1 = x[u].y >= tf;
+                    const uint32_t b0 = __ballot_sync(0xffffffffu, i0), b1 = __ballot_sync(0xffffffffu, i1);
+                    const uint32_t at = o + __popc(b0 & lt) + __popc(b1 & lt);
+                    const uint32_t q = (uint32_t)(p + 64 * u + 2 * lane);
+                    // a lane with nothing to list writes its scratch entry: no branch
+                    sh_list[i0 ? at : (uint32_t)(TR_CAP + lane)] = make_uint2(q, __float_as_uint(x[u].x));
+                    sh_list[i1 ? at + (i0 ? 1u : 0u) : (uint32_t)(TR_CAP + lane)] =
+                        make_uint2(q + 1, __float_as_uint(x[u].y));
+                    o += __popc(b0) + __popc(b1);
                 }
             }
         }
@@ -444,17 +469,11 @@ __global__ void __launch_bounds__(TR_THREADS, TR_MINB) topk_rows_kernel(const To
 
     // ---- 3. the top-K of the list
     uint32_t tau, need;
-    if (listed >= (uint32_t)K && listed <= (uint32_t)TR_CAP) {
-        if (tr_finish(sh_list, (int)listed, K, lo, hi, sh, out)) return;
-        __syncthreads();
-        // the threshold's bin is crowded (ties): exact radix levels over the list's keys
-        auto key = [&](int j) { return score_key(__uint_as_float(sh_list[j].y)); };
-        tr_select(key, (int)listed, (uint32_t)K, 0u, 0xFFFFFFFFu, sh, tau, need);
-        tr_compact([&](int j) { return make_uint2(sh_list[j].x, key(j)); }, (int)listed, tau, need, out, K, sh.ws,
-                   err);
+    if (listed >= (uint32_t)K && listed <= (uint32_t)TR_CAP && tr_finish(sh_list, (int)listed, K, lo, hi, sh, out))
         return;
-    }
-    // the list missed scores or overflowed: exact radix levels over the row's keys
+    __syncthreads();
+    // the list missed scores or overflowed, or its threshold bin is crowded (ties): exact radix levels over the
+    // row's keys
     tr_select([&](int j) { return score_key(__ldcg(row + j)); }, n, (uint32_t)K, 0u, 0xFFFFFFFFu, sh, tau, need);
     tr_compact([&](int j) { return make_uint2((uint32_t)j, score_key(__ldcg(row + j))); }, n, tau, need, out, K,
                sh.ws, err);
