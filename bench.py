@@ -118,8 +118,8 @@ class ClockSampler:
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
     BAD = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
 
-    def __init__(self, torch_device: int, period_s: float = 0.002):
-        self.samples = []
+    def __init__(self, torch_device: int, period_s: float = 0.0005):
+        self.samples = []  # (sm MHz, reason bits, host time)
         self.period = period_s
         self.ok = False
         try:
@@ -139,12 +139,21 @@ class ClockSampler:
         f = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or nv.nvmlDeviceGetCurrentClocksThrottleReasons
         return int(f(self.h))
 
+    def sample_now(self):
+        """One reading from the calling thread.  The timed loop calls this while
+        the GPU still runs the steps it has queued, so even a short timed region
+        (a few milliseconds) holds readings taken under load."""
+        if not self.ok:
+            return
+        try:
+            self.samples.append((self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM), self._reasons(),
+                                 time.perf_counter()))
+        except Exception:  # noqa: BLE001
+            pass
+
     def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append((self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM), self._reasons()))
-            except Exception:  # noqa: BLE001
-                pass
+            self.sample_now()
             time.sleep(self.period)
 
     def __enter__(self):
@@ -172,11 +181,12 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
         mhz = [s[0] for s in self.samples]
         bits = 0
-        for _, r in self.samples:
+        for _, r, _ in self.samples:
             bits |= r
         names = [n for b, n in self.REASONS.items() if bits & b]
+        t = sorted(s[2] for s in self.samples)
         return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": names,
-                "samples": len(self.samples)}
+                "samples": len(self.samples), "span_ms": round((t[-1] - t[0]) * 1e3, 3)}
 
     # reasons that explain clocks below the maximum (a power cap is kept and noted)
     EXPLAINED = {"sw_power_cap", "hw_power_brake_slowdown", "sync_boost", "applications_clocks_setting"}
@@ -315,14 +325,17 @@ def run_native(args):
         torch.cuda.synchronize()
         return ev
 
-    def timed(K):
+    def timed(K, clk):
         ev = make_events(K, 2)
         barrier()
-        for e0, e1 in ev:
+        for i, (e0, e1) in enumerate(ev):
             flush.zero_()
             e0.record(stream)
             lay.forward()
             e1.record(stream)
+            if i == 0:
+                clk.sample_now()  # the first step is running
+        clk.sample_now()  # the queued steps are still running
         barrier()
         return ev
 
@@ -337,7 +350,7 @@ def run_native(args):
     for attempt in range(2):
         clk = ClockSampler(local)
         with clk:
-            ev = timed(args.steps)
+            ev = timed(args.steps, clk)
         if not clk.rejected():
             break
     step_ms = [e0.elapsed_time(e1) for e0, e1 in ev]

@@ -47,8 +47,9 @@ def test_prefill_indexer_flops_and_topk_bytes():
 
 
 def _sampler(samples, max_mhz=1965):
+    """A sampler holding the given (MHz, reason bits) readings, 1 ms apart."""
     c = bench.ClockSampler.__new__(bench.ClockSampler)
-    c.ok, c.samples, c.max_mhz = True, samples, max_mhz
+    c.ok, c.samples, c.max_mhz = True, [(m, r, 1e-3 * i) for i, (m, r) in enumerate(samples)], max_mhz
     return c
 
 
@@ -61,6 +62,7 @@ def test_clock_record_rejects_slowdowns_and_unexplained_low_clocks():
     assert _sampler([(1200, full)] * 10).rejected()              # stuck low with no reason: a clock lock
     s = _sampler([(1965, full)] * 6 + [(1300, cap)] * 4).summary()
     assert s["sm_mhz"] == 1965 and s["reasons"] == ["sw_power_cap"] and s["samples"] == 10
+    assert s["span_ms"] == 9.0  # first to last reading
 
 
 def test_nominal_peaks_reported_beside_the_measured_ones():
