@@ -74,6 +74,8 @@ def parse_args(argv=None):
                     help="wall-clock budget of the --impl reference run")
     ap.add_argument("--prefill-only", type=int, default=0, metavar="T",
                     help="time only the prefill indexer at T queries (small cases for profiling)")
+    ap.add_argument("--with-topk", action="store_true",
+                    help="with --prefill-only: also time dsa_topk over the indexer's causal rows")
     ap.add_argument("--append-only", action="store_true",
                     help="time only the append step (dsa_append_kv), for profiling")
     ap.add_argument("--workload", choices=["decode", "cp_decode_1m"], default="decode",
@@ -1167,7 +1169,7 @@ if __name__ == "__main__":
         from long_context_sparse_02_b200 import build
         build.build()
         fl = L2Flush()
-        print(json.dumps(prefill_indexer_leg(a, fl, T=a.prefill_only, with_peak=False)))
+        print(json.dumps(prefill_indexer_leg(a, fl, T=a.prefill_only, with_peak=False, with_topk=a.with_topk)))
     elif a.append_only:
         from long_context_sparse_02_b200 import build
         build.build()
