@@ -76,6 +76,8 @@ def parse_args(argv=None):
                     help="time only the prefill indexer at T queries (small cases for profiling)")
     ap.add_argument("--with-topk", action="store_true",
                     help="with --prefill-only: also time dsa_topk over the indexer's causal rows")
+    ap.add_argument("--hybrid-only", action="store_true",
+                    help="time only the hybrid serving step (one DSA and five sliding-window layers), for profiling")
     ap.add_argument("--append-only", action="store_true",
                     help="time only the append step (dsa_append_kv), for profiling")
     ap.add_argument("--workload", choices=["decode", "cp_decode_1m"], default="decode",
@@ -588,7 +590,7 @@ def mtp_leg(args, flush, case, n=4, steps=200):
     return res
 
 
-def long_context_leg(args, flush, peaks, steps=100):
+def long_context_leg(args, flush, peaks, steps=100, which=("decode_1m", "hybrid")):
     """The layer's other decode workloads, timed like the headline (L2 flushed
     between steps, outside the events): one sequence of 1,048,576 tokens, and
     the hybrid serving step -- 64 sequences with lengths uniform in [4096,
@@ -642,6 +644,8 @@ def long_context_leg(args, flush, peaks, steps=100):
 
     res = {}
     try:
+        if "decode_1m" not in which:
+            raise LookupError
         c1 = synth.decode_1m(args.seed)
         lay = LayerOnDevice(c1, decode=True)
         ms = ms_per_step(lay.forward)
@@ -650,10 +654,14 @@ def long_context_leg(args, flush, peaks, steps=100):
                                       "roofline": hbm_roofline(decode_bytes(c1)[0], ms),
                                       "stages_us": stages(lay)})
         del lay, c1
+    except LookupError:
+        pass
     except Exception as e:  # recorded, not raised: the headline line must still print
         res["decode_1m"] = {"error": f"{type(e).__name__}: {e}"[:300]}
     torch.cuda.empty_cache()
     try:
+        if "hybrid" not in which:
+            raise LookupError
         hc = synth.hybrid_dsa(args.seed)
         lay = LayerOnDevice(hc, decode=True)
         sw = synth.swa_case(args.seed + 3, hc.seq_lens)
@@ -681,6 +689,8 @@ def long_context_leg(args, flush, peaks, steps=100):
             "group_1_dsa_5_swa": {"us_per_step": round(group_ms * 1e3, 2),
                                   "tokens_per_s": round(B / (group_ms * 1e-3), 1)}})
         del lay, rings, k0, v0
+    except LookupError:
+        pass
     except Exception as e:
         res["hybrid"] = {"error": f"{type(e).__name__}: {e}"[:300]}
     torch.cuda.empty_cache()
@@ -1170,6 +1180,11 @@ if __name__ == "__main__":
         build.build()
         fl = L2Flush()
         print(json.dumps(prefill_indexer_leg(a, fl, T=a.prefill_only, with_peak=False, with_topk=a.with_topk)))
+    elif a.hybrid_only:
+        from long_context_sparse_02_b200 import build
+        build.build()
+        fl = L2Flush()
+        print(json.dumps(long_context_leg(a, fl, load_peaks()[0], steps=a.steps, which=("hybrid",))))
     elif a.append_only:
         from long_context_sparse_02_b200 import build
         build.build()
