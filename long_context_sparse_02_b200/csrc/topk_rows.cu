@@ -395,6 +395,10 @@ __global__ void __launch_bounds__(TR_THREADS, TR_MINB) topk_rows_kernel(const To
         tr_range(lo, hi, sh.ws);
         listed = (uint32_t)n;
     } else {
+        // the whole row on its way into L2 while the threshold is chosen (one 128-byte line per prefetch): the
+        // count pass then reads it from L2
+        for (int64_t off = (int64_t)tid * 128; off < (int64_t)n * 4; off += (int64_t)TR_THREADS * 128)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char *>(row) + off));
         // this warp's range; its first loads are in flight while the threshold is chosen
         const int span = (n + 2 * TR_THREADS - 1) / (2 * TR_THREADS) * 64;
         const int wlo = min(n, warp * span), whi = min(n, wlo + span);
