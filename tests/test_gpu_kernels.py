@@ -140,6 +140,10 @@ TOPK_CASES = [
     (300, 32768, 2048, "normal"), (310, 20000, 2048, "ties"), (296, 9000, 512, "dyadic"),
     (300, 32768, 2048, "narrow"), (300, 32768, 2048, "near"), (300, 32768, 2048, "cluster"), (300, 32768, 2048, "outlier"),
     (300, 3000, 2048, "zeros"), (300, 9001, 64, "normal"),
+    # the per-row kernel's edges: every score equal and +-0 ties (the list overflows: radix fallback), rows on both
+    # sides of the 4096-entry list, K as large as the list, K = 1
+    (300, 20000, 2048, "const"), (300, 20000, 2048, "zeros"), (300, 4097, 2048, "normal"),
+    (300, 32768, 4096, "normal"), (300, 32768, 1, "dyadic"),
 ]
 
 
