@@ -76,6 +76,8 @@ def parse_args(argv=None):
                     help="time only the prefill indexer at T queries (small cases for profiling)")
     ap.add_argument("--with-topk", action="store_true",
                     help="with --prefill-only: also time dsa_topk over the indexer's causal rows")
+    ap.add_argument("--attn-only", type=int, default=0, metavar="T",
+                    help="time only the prefill attention on T queries (small cases for profiling)")
     ap.add_argument("--hybrid-only", action="store_true",
                     help="time only the hybrid serving step (one DSA and five sliding-window layers), for profiling")
     ap.add_argument("--append-only", action="store_true",
@@ -955,6 +957,50 @@ def mx_leg(args, flush, peaks, steps=100):
         return {"error": f"{type(e).__name__}: {e}"[:300]}
 
 
+def attn_only_leg(args, flush, T, L=32768, K=2048, H=128, Dqk=576, Dv=512, reps=5):
+    """dsa_sparse_attn alone on the last T prefill queries of an L-token
+    sequence, K selected causal rows each (seeded, uniform over the causal
+    prefix), 128 heads over the 576-wide latent: TFLOPS over the algorithmic
+    2 H (Dqk + Dv) K T.  For profiling the prefill attention kernel on a
+    small case."""
+    import torch
+    from long_context_sparse_02_b200 import _lib
+    g = torch.Generator(device="cuda")
+    g.manual_seed(args.seed + 3)
+    npg = L // 64
+    bt = torch.randperm(npg, generator=g, device="cuda").to(torch.int32).view(1, -1)
+    pg = _lib.paged(torch.tensor([L], dtype=torch.int32, device="cuda"), bt, npg)
+    q = (torch.randn((T, H, Dqk), device="cuda", generator=g) * 0.1).to(torch.bfloat16)
+    kv = torch.randn((npg, 64, Dqk), device="cuda", generator=g).to(torch.bfloat16)
+    gate = torch.randn((T, H), device="cuda", generator=g).to(torch.bfloat16)
+    pos = torch.arange(L - T, L, device="cuda")
+    idx = torch.sort((torch.rand((T, K), device="cuda", generator=g) * (pos[:, None] + 1).float()).long(),
+                     dim=1).values.to(torch.int32)
+    q_seq = torch.zeros(T, dtype=torch.int32, device="cuda")
+    out = torch.empty((T, H, Dv), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(max(_lib.sparse_attn_workspace_bytes(T, H, K, Dv), 1), dtype=torch.uint8, device="cuda")
+    call = lambda: _lib.sparse_attn(q, kv, pg, q_seq, idx, gate, Dqk ** -0.5, Dv, out=out, ws=ws)  # noqa: E731
+    for _ in range(2):
+        call()
+    ms = []
+    for _ in range(reps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        call()
+        e.record()
+        torch.cuda.synchronize()
+        ms.append(s.elapsed_time(e))
+    t = statistics.median(ms)
+    flops = 2.0 * H * (Dqk + Dv) * K * T  # every query has K >= 2048 causal rows to choose from
+    res = {"workload": f"prefill_attn_T{T}_of_{L}_K{K}_H{H}", "ms": round(t, 4), "algorithmic_flops": flops,
+           "tflops": round(flops / (t * 1e-3) / 1e12, 1)}
+    err = _lib.device_error(reset=True)
+    if err:
+        res["device_error"] = hex(err)
+    return res
+
+
 def tiny_layer_leg(args, flush, reps=200):
     """The tiny prefill workload (T = 1024, 4x64 indexer, K = 128, 8 heads over
     a 64-wide latent): layer latency, L2 flushed between calls."""
@@ -1180,6 +1226,10 @@ if __name__ == "__main__":
         build.build()
         fl = L2Flush()
         print(json.dumps(prefill_indexer_leg(a, fl, T=a.prefill_only, with_peak=False, with_topk=a.with_topk)))
+    elif a.attn_only:
+        from long_context_sparse_02_b200 import build
+        build.build()
+        print(json.dumps(attn_only_leg(a, L2Flush(), a.attn_only)))
     elif a.hybrid_only:
         from long_context_sparse_02_b200 import build
         build.build()
