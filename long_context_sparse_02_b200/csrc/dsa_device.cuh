@@ -326,6 +326,35 @@ __device__ __forceinline__ void st_global_if(float *addr, float v, bool pred) {
                  "f"(v), "r"((uint32_t)pred)
                  : "memory");
 }
+__device__ __forceinline__ void st_global_if(int32_t *addr, uint32_t v, bool pred) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %2, 0;\n\t@p st.global.b32 [%0], %1;\n\t}" ::"l"(addr),
+                 "r"(v), "r"((uint32_t)pred)
+                 : "memory");
+}
+__device__ __forceinline__ void st_global_if(uint2 *addr, uint2 v, bool pred) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %3, 0;\n\t@p st.global.v2.b32 [%0], {%1, %2};\n\t}" ::"l"(addr),
+                 "r"(v.x), "r"(v.y), "r"((uint32_t)pred)
+                 : "memory");
+}
+__device__ __forceinline__ void st_shared_if(uint32_t *addr, uint32_t v, bool pred) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %2, 0;\n\t@p st.shared.b32 [%0], %1;\n\t}" ::"r"(
+                     smem_u32(addr)),
+                 "r"(v), "r"((uint32_t)pred)
+                 : "memory");
+}
+// *addr += 1 where pred holds (shared memory; global memory relaxed at device scope)
+__device__ __forceinline__ void inc_shared_if(uint32_t *addr, bool pred) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t@p red.shared.add.u32 [%0], 1;\n\t}" ::"r"(
+                     smem_u32(addr)),
+                 "r"((uint32_t)pred)
+                 : "memory");
+}
+__device__ __forceinline__ void inc_global_if(uint32_t *addr, bool pred) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t@p red.relaxed.gpu.global.add.u32 [%0], 1;\n\t}" ::"l"(
+                     addr),
+                 "r"((uint32_t)pred)
+                 : "memory");
+}
 
 // ---- programmatic dependent launch -----------------------------------------------
 // A kernel launched with programmatic stream serialization may start before

@@ -196,24 +196,6 @@ static_assert(LBINS == 2 * CT_THREADS, "two bins per thread");
 // 22 list overflow; 24,25 above-b keys / bin-b keys of earlier CTAs;
 // 32..47 bin-b keys of earlier CTAs, per CTA rank
 
-// Predicated forms (one instruction under a predicate rather than a branch):
-// a global or shared store, and a shared-memory increment, where c holds.
-__device__ __forceinline__ void st_global_pred(bool c, int32_t *p, uint32_t v) {
-    asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t@q st.global.b32 [%1], %2;\n\t}" ::"r"((uint32_t)c),
-                 "l"(p), "r"(v)
-                 : "memory");
-}
-__device__ __forceinline__ void st_shared_pred(bool c, uint32_t *p, uint32_t v) {
-    asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t@q st.shared.b32 [%1], %2;\n\t}" ::"r"((uint32_t)c),
-                 "r"(smem_u32(p)), "r"(v)
-                 : "memory");
-}
-__device__ __forceinline__ void inc_shared_pred(bool c, uint32_t *p) {
-    asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t@q red.shared.add.u32 [%1], 1;\n\t}" ::"r"((uint32_t)c),
-                 "r"(smem_u32(p))
-                 : "memory");
-}
-
 __device__ __forceinline__ int linear_bin(float x, float lo, float scale) {
     const float y = __fmul_rn(__fsub_rn(x, lo), scale);
     return min(LBINS - 1, __float2int_rz(y));
@@ -557,9 +539,9 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
                     const float x = xv[st][k];
                     const uint32_t key = score_key(x);
                     const int fbn = linear_bin(x, xlo, fscale);  // meaningful only for keys of bin B
-                    inc_shared_pred(b && (key >> SCORE_HIST_SHIFT) == B, lhist + (fbn > 0 ? fbn : 0));
-                    st_shared_pred(b && so < (uint32_t)WCAP, wl + (so < (uint32_t)WCAP ? so : 0u), (uint32_t)(i0 + k));
-                    st_shared_pred(b && so < (uint32_t)WCAP, wk + (so < (uint32_t)WCAP ? so : 0u), key);
+                    inc_shared_if(lhist + (fbn > 0 ? fbn : 0), b && (key >> SCORE_HIST_SHIFT) == B);
+                    st_shared_if(wl + (so < (uint32_t)WCAP ? so : 0u), (uint32_t)(i0 + k), b && so < (uint32_t)WCAP);
+                    st_shared_if(wk + (so < (uint32_t)WCAP ? so : 0u), key, b && so < (uint32_t)WCAP);
                     so += b ? 1u : 0u;
                 }
                 cnt += stot;
@@ -726,7 +708,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) topk_cluster_kernel(const TopkA
                     const uint32_t mg = gcur + __popc(gm & lt), me = ecur + __popc(em & lt);
                     const bool keep = gt || (eq && me < need);
                     const uint32_t slot = mg + min(me, need);
-                    st_global_pred(keep && slot < Ku, out + slot, (uint32_t)(s0 + (int)(j < wn ? wl[j] : 0u)));
+                    st_global_if(out + slot, (uint32_t)(s0 + (int)(j < wn ? wl[j] : 0u)), keep && slot < Ku);
                     if (keep && slot >= Ku) record_error(err, DSA_DEVERR_SHAPE);
                     gcur += __popc(gm);
                     ecur += __popc(em);

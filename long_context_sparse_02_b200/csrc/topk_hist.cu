@@ -131,26 +131,6 @@ __device__ __forceinline__ void ht_pick_smem(const uint32_t *hist, uint32_t rema
 // pass counts each segment's kept candidates, one exchange gives every
 // segment its offsets, a second pass writes.  entry(j) returns (position,
 // key); position PAD marks an entry to skip.  ws: 2 * HT_WARPS words.
-// Predicated forms (one instruction under a predicate rather than a branch):
-// *p = v, and *p += 1 (relaxed, device scope), where c holds.
-__device__ __forceinline__ void ht_st_if(bool c, int32_t *p, uint32_t v) {
-    asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t@q st.global.b32 [%1], %2;\n\t}" ::"r"((uint32_t)c),
-                 "l"(p), "r"(v)
-                 : "memory");
-}
-__device__ __forceinline__ void ht_st2_if(bool c, uint2 *p, uint2 v) {
-    asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t@q st.global.v2.b32 [%1], {%2, %3};\n\t}" ::"r"(
-                     (uint32_t)c),
-                 "l"(p), "r"(v.x), "r"(v.y)
-                 : "memory");
-}
-__device__ __forceinline__ void ht_inc_if(bool c, uint32_t *p) {
-    asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t@q red.relaxed.gpu.global.add.u32 [%1], 1;\n\t}" ::"r"(
-                     (uint32_t)c),
-                 "l"(p)
-                 : "memory");
-}
-
 template <int E, typename Entry>
 __device__ __forceinline__ void ht_compact(Entry entry, int64_t count, uint32_t tau, uint32_t need, int32_t *out,
                                            int K, uint32_t *ws, uint32_t *err) {
@@ -197,7 +177,7 @@ __device__ __forceinline__ void ht_compact(Entry entry, int64_t count, uint32_t 
         for (int i = 0; i < E; ++i) {
             const bool keep = gt[i] || (eq[i] && me < need);
             const uint32_t slot = mg + min(me, need);
-            ht_st_if(keep && slot < (uint32_t)K, out + slot, v[i].x);
+            st_global_if(out + slot, v[i].x, keep && slot < (uint32_t)K);
             if (keep && slot >= (uint32_t)K) record_error(err, DSA_DEVERR_SHAPE);
             mg += gt[i], me += eq[i];
         }
@@ -325,7 +305,7 @@ __global__ void __launch_bounds__(HT_THREADS, 1) topk_hist_kernel(const TopkArgs
                 m[g] |= (in ? 1u : 0u) << k;
                 n_above += in && cb > B;
                 n_in += in && cb == B;
-                ht_inc_if(in && cb == B, frow + ((key >> 10) & (FINE_BINS - 1)));
+                inc_global_if(frow + ((key >> 10) & (FINE_BINS - 1)), in && cb == B);
             }
             const uint32_t cnt = __popc(m[g]);
             const uint32_t incl = warp_incl_scan(cnt);
@@ -348,7 +328,7 @@ __global__ void __launch_bounds__(HT_THREADS, 1) topk_hist_kernel(const TopkArgs
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const bool b = ((m[g] >> k) & 1u) != 0;
-                ht_st2_if(b, region + o, make_uint2((uint32_t)(p0 + k), score_key(x[g][k])));
+                st_global_if(region + o, make_uint2((uint32_t)(p0 + k), score_key(x[g][k])), b);
                 o += b ? 1u : 0u;
             }
         }

@@ -267,13 +267,6 @@ __device__ __forceinline__ void tr_load_any(const float *row, int p, int hi, flo
     else tr_load<false>(row, p, hi, x);
 }
 
-// *p = v where c holds, as one predicated store rather than a branch.
-__device__ __forceinline__ void tr_store_if(bool c, int32_t *p, uint32_t v) {
-    asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %0, 0;\n\t@q st.global.b32 [%1], %2;\n\t}" ::"r"((uint32_t)c),
-                 "l"(p), "r"(v)
-                 : "memory");
-}
-
 // Top-K of the listed entries (K <= listed <= TR_CAP, every score >= lo):
 // the histogram over [lo, hi] (scores above hi count in the top bin), then
 // the two passes.  Returns false, having written nothing, when the
@@ -347,7 +340,7 @@ __device__ __forceinline__ bool tr_finish(uint2 *list, int listed, int K, float 
         const bool keep = bn > F || (bn == F && (ex & TR_MARK));
         const uint32_t km = __ballot_sync(0xffffffffu, keep);
         const uint32_t slot = base + __popc(km & lt);
-        tr_store_if(keep && slot < (uint32_t)K, out + slot, ex & TR_POS);
+        st_global_if(out + slot, ex & TR_POS, keep && slot < (uint32_t)K);
         base += __popc(km);
     }
     return true;
