@@ -14,9 +14,11 @@
 //      the bin, in a 256-bin histogram over the sample's range, that holds
 //      the sample score whose rank is the expected rank of the K-th score
 //      plus four standard deviations;
-//   2. each warp counts its scores >= tf, the counts give each warp its
-//      offset, and a second pass over the warp's range (now in L2) lists
-//      them as (position, score) in position order into shared memory;
+//   2. the row, sent into L2 by prefetches at the CTA's start (while step 1
+//      runs), is read twice from there: each warp counts its scores >= tf,
+//      the counts give each warp its offset, and a second pass over the
+//      warp's range lists them as (position, score) in position order into
+//      shared memory;
 //   3. a 1024-bin histogram of the listed scores over [tf, sample maximum]
 //      gives the bin F of the K-th score; one pass over the list counts the
 //      entries above F and collects F's few entries, one warp ranks those
