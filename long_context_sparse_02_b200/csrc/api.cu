@@ -389,7 +389,7 @@ dsa_status dsa_layer_forward_profiled(const dsa_layer_args *a, void *ws, size_t 
 
 int32_t dsa_layer_kernel_launches(const dsa_layer_args *a) {
     if (!a || a->T <= 0 || a->max_len < 1) return 0;
-    return 1 + (hist_mode(a) ? 1 : topk_kernel_launches(a->T, a->max_len)) + attn_kernel_launches(a->T, a->K, a->Dv);
+    return 1 + (hist_mode(a) ? 1 : topk_kernel_launches(a->T, a->K, a->max_len)) + attn_kernel_launches(a->T, a->K, a->Dv);
 }
 
 dsa_status dsa_append_kv(const uint16_t *k_new, float k_scale, const uint16_t *latent_new, const int32_t *tok_seq,

@@ -91,7 +91,7 @@ struct TopkArgs {
     uint32_t *hist;
 };
 size_t topk_workspace_bytes(int32_t R, int32_t K, int32_t max_row_len);
-int topk_kernel_launches(int32_t R, int32_t max_row_len);
+int topk_kernel_launches(int32_t R, int32_t K, int32_t max_row_len);
 // Few rows that each fit one large thread-block cluster (10 or 16 CTAs, all
 // clusters resident at once): the cluster kernel, which also reads the
 // indexer's histogram, selects faster than the single-launch list-and-ticket
@@ -112,10 +112,10 @@ HistTopkPlan topk_hist_plan(int32_t R, int32_t max_row_len);
 size_t topk_hist_workspace_bytes(int32_t R, int32_t max_row_len);
 int64_t topk_hist_zero_words(int32_t R);
 dsa_status launch_topk_hist(const TopkArgs &a, cudaStream_t st);
-// Many rows (R >= 2 x SMs), each at most 32768 keys long: one 512-thread CTA
-// per row lists its keys at or above the threshold's coarse bin in shared
-// memory and selects from there.  No workspace.
-bool topk_rows_eligible(int32_t R, int32_t max_row_len);
+// Many rows (R >= 2 x SMs), each at most 32768 keys long, K <= 2048: one
+// 256-thread CTA per row lists its likely candidates in shared memory and
+// selects from there.  No workspace.
+bool topk_rows_eligible(int32_t R, int32_t K, int32_t max_row_len);
 dsa_status launch_topk_rows(const TopkArgs &a, cudaStream_t st);
 
 // ---- gated sparse attention ----------------------------------------------------

@@ -1300,7 +1300,7 @@ dsa_status launch_cluster(const TopkArgs &a, const ClusterPlan &cp, cudaStream_t
 size_t topk_workspace_bytes(int32_t R, int32_t K, int32_t max_row_len) {
     (void)K;
     const DeviceInfo *dev = current_device();
-    if (dev && (topk_rows_eligible(R, max_row_len) || cluster_plan(R, max_row_len, dev).cl > 0)) return 0;
+    if (dev && (topk_rows_eligible(R, K, max_row_len) || cluster_plan(R, max_row_len, dev).cl > 0)) return 0;
     const int nch = (max_row_len + CHUNK - 1) / CHUNK;
     return align_up(multi_zero_bytes(R) + (size_t)R * nch * 2 * 4, 256);
 }
@@ -1310,16 +1310,16 @@ bool topk_prefers_cluster(int32_t R, int32_t max_row_len) {
     return dev && cluster_plan(R, max_row_len, dev).cl >= 10;
 }
 
-int topk_kernel_launches(int32_t R, int32_t max_row_len) {
+int topk_kernel_launches(int32_t R, int32_t K, int32_t max_row_len) {
     const DeviceInfo *dev = current_device();
-    return (dev && (topk_rows_eligible(R, max_row_len) || cluster_plan(R, max_row_len, dev).cl > 0)) ? 1 : 5;
+    return (dev && (topk_rows_eligible(R, K, max_row_len) || cluster_plan(R, max_row_len, dev).cl > 0)) ? 1 : 5;
 }
 
 dsa_status launch_topk(const TopkArgs &a, cudaStream_t st) {
     const DeviceInfo *dev = current_device();
     if (!dev) return DSA_ERR_CUDA;
     if (a.R == 0) return DSA_OK;
-    if (!a.hist && topk_rows_eligible(a.R, a.max_row_len) && !(reinterpret_cast<uintptr_t>(a.scores) & 15u) &&
+    if (!a.hist && topk_rows_eligible(a.R, a.K, a.max_row_len) && !(reinterpret_cast<uintptr_t>(a.scores) & 15u) &&
         !(a.ld & 3))
         return launch_topk_rows(a, st);
     const ClusterPlan cp = cluster_plan(a.R, a.max_row_len, dev);

@@ -480,9 +480,10 @@ __global__ void __launch_bounds__(TR_THREADS, TR_MINB) topk_rows_kernel(const To
 
 }  // namespace
 
-bool topk_rows_eligible(int32_t R, int32_t max_row_len) {
+bool topk_rows_eligible(int32_t R, int32_t K, int32_t max_row_len) {
+    // K up to half the list: a larger K would overflow it on most rows (the radix fallback every time)
     const DeviceInfo *dev = current_device();
-    return dev && R >= 2 * dev->sm_count && max_row_len <= TR_MAXN;
+    return dev && R >= 2 * dev->sm_count && max_row_len <= TR_MAXN && K <= TR_CAP / 2;
 }
 
 dsa_status launch_topk_rows(const TopkArgs &a, cudaStream_t st) {
